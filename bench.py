@@ -1,0 +1,434 @@
+#!/usr/bin/env python
+"""Decode throughput of the Qwen2-1.5B-shaped decoder on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One JSON line on stdout (rank 0).  A "step" is one greedy decode step of the
+whole hot path (embedding, 28 decoder layers, final norm, lm_head, argmax)
+for every sequence of the batch.  Workload (default): the full 28-layer
+Qwen2-1.5B shape, random-init bf16 weights, batch 1, a 512-token prompt of
+uniform random ids prefilled first (timed separately), then the timed decode
+steps (context 512 + warmup + steps).  Per step the kernels stream all
+3.09 GB of weights, far more than the 126 MB L2, so no L2 flush is needed.
+Extra keys report batch 64 at 4096 context (KV filled with N(0,1)), the
+prefill, per-kernel times and the CPU oracle baseline.
+
+Multi-GPU: replicas (`--gpus N` under torchrun): every rank decodes its own
+sequences, no data-path collective; the time is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "decode tok/s (Qwen2-1.5B shape, bf16, B=1/64); achieved HBM GB/s vs peak"
+WORKLOAD = "qwen2-1.5b-b1-prompt512-decode128"
+WORKLOAD_B64 = "qwen2-1.5b-b64-ctx4096-decode32"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+# ------------------------------------------------------------ distributed
+
+class Dist:
+    def __init__(self):
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+
+    def init(self, use_cuda: bool):
+        if self.world > 1:
+            import torch.distributed as dist
+            kw = dict(timeout=datetime.timedelta(seconds=300))
+            if use_cuda:
+                torch.cuda.set_device(self.local)
+                dist.init_process_group("nccl", device_id=torch.device(f"cuda:{self.local}"), **kw)
+            else:
+                dist.init_process_group("gloo", **kw)
+            self.pg = dist
+        elif use_cuda:
+            torch.cuda.set_device(self.local)
+
+    def barrier(self):
+        if self.pg:
+            self.pg.barrier()
+
+    def max(self, x: float) -> float:
+        if not self.pg:
+            return x
+        dev = f"cuda:{self.local}" if torch.cuda.is_available() else "cpu"
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+# ------------------------------------------------------------------ clocks
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during timed work."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.idx)], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        rows = []
+        if self.path and os.path.exists(self.path):
+            for line in open(self.path):
+                f = [x.strip() for x in line.split(",")]
+                if len(f) >= 8:
+                    rows.append(f)
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------- byte accounting
+
+def layer_weight_bytes(s) -> int:
+    es = 2 if s.dtype == "bf16" else 4
+    qkvd = s.q_dim + 2 * s.kv_dim
+    return es * (qkvd * s.hidden + qkvd + s.hidden * s.q_dim + 3 * s.intermediate * s.hidden + 2 * s.hidden)
+
+
+def decode_step_bytes(s, batch: int, ctx: float) -> float:
+    """Algorithmic HBM bytes of one decode step: every weight once (the
+    embedding table only for the rows read), the KV of every visible position
+    of every sequence read once, the new K/V written."""
+    es = 2 if s.dtype == "bf16" else 4
+    kv_per_pos = 2 * s.n_layers * s.kv_dim * es
+    w = s.n_layers * layer_weight_bytes(s) + es * (s.vocab * s.hidden + s.hidden)
+    return w + batch * (ctx + 1) * kv_per_pos + batch * s.hidden * es
+
+
+def kernel_src_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "qwen2_decode_step_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        h.update(open(os.path.join(csrc, fn), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """Per-launch DRAM bytes from a committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    e = d.get(f"{kernel}@{workload}")
+    if not e or e.get("src_hash") != kernel_src_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# --------------------------------------------------------------- oracle leg
+
+def oracle_decode_sample(max_seconds: float, max_substeps: int, seed: int = 1003):
+    """Times the CPU oracle on a bounded sample of the B=1 decode step of the
+    full Qwen2-1.5B shape at context 512: a sub-step is one full-size decoder
+    layer (decode of one token against 512 cached positions) plus 1/28 of the
+    lm_head rows; 28 sub-steps are one token's work.  Returns (tok/s, sample
+    description, sub-steps run)."""
+    import oracle
+    shape = synth.QWEN2_1P5B_ONE_LAYER
+    w = {k: synth.weight(shape, k[0], k[1], seed) for k in shape.weight_shapes()
+         if k[0] not in ("embed", "lm_head")}
+    om = oracle.OracleModel(shape, max_seq=600)
+    om.load(w)
+    k, v = synth.kv_fill(shape, 512, seed, 0, 0)
+    ok, ov = om.kv(0, 0)
+    ok[:512] = k
+    ov[:512] = v
+    x = synth.hidden_input(shape, 1, seed)
+    rows = (synth.QWEN2_1P5B.vocab + 27) // 28
+    lm = synth.normal((rows, shape.hidden), 0.02, 99, "bf16")
+    h = synth.normal((1, shape.hidden), 1.0, 98, "bf16")
+    spent, n = 0.0, 0
+    while n < max_substeps and (spent < max_seconds or n == 0):
+        om.set_len(0, 512)
+        t0 = time.perf_counter()
+        om.forward_hidden(0, x)
+        oracle.linear(h, lm, None, out_dtype=torch.float32)
+        spent += time.perf_counter() - t0
+        n += 1
+    per_token = spent / n * 28
+    desc = (f"{n} sub-steps; each = one full-size Qwen2-1.5B decoder layer decoding 1 token at "
+            f"context 512 + lm_head GEMV over {rows} of {synth.QWEN2_1P5B.vocab} vocab rows (1/28); "
+            f"28 sub-steps = one decode step (tok/s = 1 / (28 x mean sub-step time))")
+    return 1.0 / per_token, desc, n
+
+
+def run_reference(args, dist: Dist):
+    """The oracle arm: the plain CPU oracle, as it stands, on the host cores."""
+    dist.init(use_cuda=False)
+    if dist.rank != 0:
+        dist.close()
+        return
+    import oracle
+    oracle.lib()
+    # warm-up sub-steps (untimed), then K timed sub-steps bounded to a few minutes
+    oracle_decode_sample(0.0, max(1, min(args.warmup, 3)))
+    t0 = time.perf_counter()
+    tps, desc, n = oracle_decode_sample(max_seconds=min(120.0, 1.5 * args.steps),
+                                        max_substeps=args.steps)
+    wall = time.perf_counter() - t0
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tps, "unit": "tok/s", "n_gpus": args.gpus,
+        "steps": n, "warmup": args.warmup, "ms_per_step": 1000.0 / tps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64 (bf16 storage)", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "batch": 1, "context": 512, "sampled": True},
+        "cpu_baseline": {"value": tps, "unit": "tok/s", "cores": 1, "kind": "oracle", "sample": desc},
+        "e2e": {"value": tps, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "wall_s": wall,
+    }
+    print(json.dumps(line), flush=True)
+    dist.close()
+
+
+# ----------------------------------------------------------------- our arm
+
+def cuda_time(fn, n: int) -> float:
+    """ms of n calls of fn, CUDA events on the current stream."""
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    s.record()
+    for _ in range(n):
+        fn()
+    e.record()
+    torch.cuda.synchronize()
+    return s.elapsed_time(e)
+
+
+def run_ours(args, dist: Dist):
+    import qwen2_decode_step_b200 as q2
+    dist.init(use_cuda=True)
+    dev = torch.cuda.current_device()
+    shape = synth.QWEN2_1P5B
+    wl = synth.WORKLOADS[WORKLOAD]
+    seed = wl["seed"] + 100 * dist.rank
+    prompt_len = wl["prompt"]
+    b64 = not args.no_b64
+    max_batch = 64 if b64 else 1
+    past64 = synth.WORKLOADS[WORKLOAD_B64]["past"]
+    max_seq = max(prompt_len + args.warmup + args.steps + 64, (past64 + args.b64_steps + 16) if b64 else 0)
+    model = q2.Model(shape, max_seq=max_seq, max_batch=max_batch)
+    for key in shape.weight_shapes():  # drawn on the GPU tensor by tensor, copied in, freed
+        t = synth.weight(shape, key[0], key[1], seed, device="cuda")
+        model.load_weight(key[0], key[1], t)
+        del t
+    torch.cuda.synchronize()
+
+    # ---- prefill (load and generate are timed apart)
+    ids = synth.prompt_ids(shape, prompt_len, seed, device="cuda")
+    model.prefill(ids, [prompt_len])
+    model.reset_kv()
+    torch.cuda.synchronize()
+    pre_ms = cuda_time(lambda: model.prefill(ids, [prompt_len]), 1)
+    model.reset_kv()
+    nxt = model.prefill(ids, [prompt_len])
+
+    clocks = Clocks(dev)
+    # ---- B = 1 decode: warm-up, then K timed steps
+    bufs = [nxt.clone(), torch.empty_like(nxt)]
+    for i in range(args.warmup):
+        model.decode_step(bufs[i % 2], out=bufs[(i + 1) % 2])
+    cur = args.warmup % 2
+    clocks.start()
+    dist.barrier()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for i in range(args.steps):
+        model.decode_step(bufs[(cur + i) % 2], out=bufs[(cur + i + 1) % 2])
+    e.record()
+    torch.cuda.synchronize()
+    dist.barrier()
+    ms = dist.max(s.elapsed_time(e))
+    ms_step = ms / args.steps
+    ctx_mean = prompt_len + args.warmup + (args.steps - 1) / 2.0
+    step_bytes = decode_step_bytes(shape, 1, ctx_mean)
+
+    # ---- per-kernel device times inside the same decode step (instrumented replay)
+    last = bufs[(cur + args.steps) % 2]
+    ktimes, kernels_per_step = model.time_kernels(last, steps=min(args.steps, 20))
+
+    # ---- e2e: the public host-buffer entry point, H2D ids + D2H next each step
+    ids_h = torch.empty(1, dtype=torch.int64).pin_memory()
+    out_h = torch.empty(1, dtype=torch.int64).pin_memory()
+    ids_h.copy_(last.cpu())
+    for _ in range(3):
+        model.decode_step_host(ids_h, out_h)
+        ids_h.copy_(out_h)
+    dist.barrier()
+
+    def e2e_step():
+        model.decode_step_host(ids_h, out_h)
+        ids_h.copy_(out_h)
+    e2e_n = max(1, min(args.steps, 100))
+    e2e_ms = dist.max(cuda_time(e2e_step, e2e_n)) / e2e_n
+
+    # ---- batch 64 at 4096 context (KV N(0,1), kernel-only fill)
+    b64_line = None
+    if b64:
+        B = 64
+        for l in range(shape.n_layers):
+            for b in range(B):
+                k, v = synth.kv_fill(shape, past64, seed, l, b, device="cuda")
+                gk, gv = model.kv_cache(l, b)
+                gk[:, :past64].copy_(k.permute(1, 0, 2))
+                gv[:, :past64].copy_(v.permute(1, 0, 2))
+        torch.cuda.synchronize()
+        for b in range(B):
+            model.set_seq_len(b, past64)
+        ids64 = synth.uniform_ids(B, shape.vocab, seed + 7, device="cuda")
+        b64bufs = [ids64, torch.empty_like(ids64)]
+        for i in range(3):
+            model.decode_step(b64bufs[i % 2], out=b64bufs[(i + 1) % 2])
+        n64 = args.b64_steps
+        dist.barrier()
+        ms64 = dist.max(cuda_time_b64(model, b64bufs, n64)) / n64
+        ctx64 = past64 + 3 + (n64 - 1) / 2.0
+        bytes64 = decode_step_bytes(shape, B, ctx64)
+        b64_line = {"workload": WORKLOAD_B64, "batch": B, "value": B * dist.world / (ms64 / 1e3),
+                    "unit": "tok/s", "ms_per_step": ms64, "steps": n64,
+                    "achieved_gbs": bytes64 / (ms64 / 1e3) / 1e9, "bytes_per_step": bytes64}
+    clk = clocks.stop()
+
+    pk, pk_kind = peaks()
+    hbm = float(pk["hbm_gbs"])
+    gu_ms, gu_n = ktimes["gate_up"]
+    gu_bytes = 2 * shape.intermediate * shape.hidden * 2 + shape.hidden * 2 + 2 * shape.intermediate * 2
+    achieved = gu_bytes / (gu_ms / 1e3) / 1e9 if gu_ms > 0 else None
+    line = {
+        "metric": METRIC,
+        "value": 1 * dist.world / (ms_step / 1e3),
+        "unit": "tok/s",
+        "n_gpus": dist.world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (random-init bf16 weights, uniform random prompt ids)",
+        "config": {"workload": WORKLOAD, "batch": 1, "prompt": prompt_len,
+                   "context": f"{prompt_len + args.warmup}..{prompt_len + args.warmup + args.steps}",
+                   "l2": "no flush: each step streams 3.09 GB of weights (> 126 MB L2)",
+                   "parallelism": f"replicas x{dist.world}"},
+        "step_roofline": {"bytes_per_step": step_bytes, "achieved_gbs": step_bytes / (ms_step / 1e3) / 1e9,
+                          "peak_gbs": hbm, "frac": step_bytes / (ms_step / 1e3) / 1e9 / hbm,
+                          "peak_kind": pk_kind},
+        "roofline": {"kernel": "gate_up", "bound": "hbm", "achieved": achieved, "peak": hbm,
+                     "unit": "GB/s", "frac": (achieved / hbm) if achieved else None,
+                     "traffic": recorded_traffic("gate_up", WORKLOAD),
+                     "bytes_per_launch": gu_bytes, "mean_launch_ms": gu_ms, "peak_kind": pk_kind},
+        "kernels_ms": {k: {"mean_ms": round(v[0], 5), "per_step": v[1]} for k, v in ktimes.items() if v[1]},
+        "gpu_launches": kernels_per_step * args.steps,
+        "kernels_per_step": kernels_per_step,
+        "prefill": {"tokens": prompt_len, "ms": pre_ms, "tok_s": prompt_len / (pre_ms / 1e3)},
+        "e2e": {"value": 1 * dist.world / (e2e_ms / 1e3), "unit": "tok/s", "h2d_bytes_per_step": 8,
+                "d2h_bytes_per_step": 8, "ms_per_step": e2e_ms,
+                "api": "q2_model_decode_step_host (pinned host ids -> host next)"},
+        "b64": b64_line,
+        "clocks": clk,
+    }
+    model.close()
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        tps, desc, n = oracle_decode_sample(max_seconds=args.cpu_seconds, max_substeps=10_000)
+        line["cpu_baseline"] = {"value": tps, "unit": "tok/s", "cores": 1, "kind": "oracle",
+                                "sample": desc}
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+    dist.close()
+
+
+def cuda_time_b64(model, bufs, n):
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    s.record()
+    for i in range(n):
+        model.decode_step(bufs[i % 2], out=bufs[(i + 1) % 2])
+    e.record()
+    torch.cuda.synchronize()
+    return s.elapsed_time(e)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--b64-steps", type=int, default=32)
+    ap.add_argument("--no-b64", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    dist = Dist()
+    if args.impl == "reference":
+        run_reference(args, dist)
+    else:
+        run_ours(args, dist)
+
+
+if __name__ == "__main__":
+    main()

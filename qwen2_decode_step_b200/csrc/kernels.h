@@ -1,0 +1,73 @@
+// kernels.h -- internal launchers shared by the C-ABI entry points and the
+// model runtime.  Every launcher enqueues on `st` and returns a status; none
+// synchronises.  `pdl` requests programmatic dependent launch (the kernel
+// then waits for its predecessor with griddepcontrol.wait before touching
+// any activation).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/q2.h"
+
+namespace q2 {
+
+size_t dtype_size(int dtype);
+
+q2_status launch_add(void* c, const void* a, const void* b, size_t n, int dtype, cudaStream_t st);
+q2_status launch_swiglu(void* out, const void* gate, const void* up, size_t n, int dtype,
+                        cudaStream_t st);
+// out[t, :] = gate_up[t, 0:I] -> silu, times gate_up[t, I:2I]; rows of stride 2I.
+q2_status launch_swiglu_rows(void* out, const void* gate_up, int T, int I, int dtype,
+                             cudaStream_t st, bool pdl);
+q2_status launch_embedding(void* out, const int64_t* ids, const void* table, size_t ntok,
+                           size_t vocab, size_t d, int dtype, int* err_flag, cudaStream_t st,
+                           bool pdl);
+// residual += y (rounded; y may be NULL), h = rms_norm(residual) * w.  h may be NULL
+// (then only the add happens).
+q2_status launch_add_rms_norm(void* residual, const void* y, void* h, const void* w, size_t M,
+                              size_t d, float eps, int dtype, cudaStream_t st, bool pdl);
+q2_status launch_rms_norm(void* out, const void* in, const void* w, size_t M, size_t d, float eps,
+                          int dtype, cudaStream_t st);
+q2_status launch_rope(void* out, const void* in, const int64_t* pos, size_t ntok, size_t nhead,
+                      size_t hd, float theta, int dtype, cudaStream_t st);
+q2_status launch_rearrange(void* out, const void* in, int ndim, const int64_t* shape,
+                           const int64_t* out_strides, const int64_t* in_strides, size_t elem_size,
+                           cudaStream_t st);
+// Two-pass argmax.  part_val/part_idx hold rows * parts partials (parts from
+// argmax_parts()).
+int argmax_parts(size_t rows, size_t n);
+q2_status launch_argmax(int64_t* idx, void* val, const void* x, size_t rows, size_t n, int dtype,
+                        float* part_val, int64_t* part_idx, int parts, cudaStream_t st, bool pdl);
+
+// ------------------------------------------------------------------ linear
+// out[M, N] (out_dtype) = in[M, K] . W[N, K]^T + b (dtype).
+q2_status launch_linear(void* out, const void* in, const void* w, const void* b, int M, int N,
+                        int K, int dtype, int out_dtype, cudaStream_t st, bool pdl);
+
+// --------------------------------------------------------------- attention
+struct AttnRows {
+  const void* q;
+  long long q_row_stride;  // elements between query rows
+  const void* k;
+  const void* v;
+  long long kv_seq_stride;   // elements between sequences
+  long long kv_tok_stride;   // elements between positions
+  long long kv_head_stride;  // elements between kv heads
+  void* out;
+  long long out_row_stride;
+  int rows, nh, nkv, hd;
+  // visible keys of query row r: base + row_step * r + (lens ? lens[seq(r)] : 0),
+  // with seq(r) = seq_is_row ? r : fixed_seq.
+  int base, row_step;
+  const int* lens;
+  int seq_is_row, fixed_seq;
+  float scale;
+};
+// Split count for a given problem (decode: enough CTAs for the machine).
+int attn_splits(int rows, int nkv, int max_keys);
+size_t attn_scratch_bytes(int rows, int nh, int hd, int nsplit);
+q2_status launch_attention(const AttnRows& a, int nsplit, void* scratch, int dtype,
+                           cudaStream_t st, bool pdl);
+
+}  // namespace q2

@@ -1,0 +1,798 @@
+// model.cu -- the Qwen2-style decoder runtime behind q2_model_*: weights, KV
+// cache and every activation buffer allocated once at create time (LLAISYS
+// final report, section 3.3, item 4: per-token buffer allocation and
+// per-call handle creation were the cost that dominated), prefill in
+// chunks, and a decode step captured once per batch size as a CUDA graph
+// whose kernels chain with programmatic dependent launch.
+//
+// Layer order (the Qwen2 decoder the report runs on the GPU, section 3.2,
+// fourth layer): RMSNorm -> q/k/v linear (+bias) -> RoPE -> KV write-back ->
+// causal GQA attention -> o linear -> residual add + RMSNorm -> gate/up
+// linear -> SwiGLU -> down linear -> residual add (+ next RMSNorm).  Final:
+// RMSNorm -> lm_head (fp32 logits) -> argmax.
+#include <math.h>
+
+#include <map>
+#include <vector>
+
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace q2;
+
+struct LayerW {
+  void* in_norm;
+  void* wqkv;  // [nh*hd + 2*nkv*hd, H]: q rows, then k rows, then v rows
+  void* bqkv;  // [nh*hd + 2*nkv*hd]
+  void* wo;    // [H, nh*hd]
+  void* post_norm;
+  void* wgu;  // [2I, H]: gate rows, then up rows
+  void* wd;   // [H, I]
+};
+
+// Event pairs around kernel-class instances, for q2_model_time_kernels.
+struct KTiming {
+  std::vector<cudaEvent_t> ev;  // 2 per mark: begin, end
+  std::vector<int> cls;
+  size_t used = 0;
+  cudaGraphExec_t exec = nullptr;
+  int kernels = 0;
+};
+
+struct q2_model {
+  q2_meta m{};
+  int device = 0;
+  int dt = Q2_BF16;
+  size_t es = 2;
+  int qd = 0, kd = 0, qkvd = 0, chunk = 0, tmax = 0;
+
+  void* wbuf = nullptr;
+  void* embed = nullptr;
+  void* lm_head = nullptr;
+  void* final_norm = nullptr;
+  std::vector<LayerW> layers;
+
+  void* kc = nullptr;  // [L][Bmax][nkv][max_seq][hd]
+  void* vc = nullptr;
+  long long kv_seq_stride = 0, kv_layer_stride = 0;
+  int* d_len = nullptr;
+  std::vector<int> h_len;
+
+  void *x = nullptr, *h = nullptr, *qkv = nullptr, *att = nullptr, *o = nullptr, *gu = nullptr,
+       *s = nullptr;
+  float* logits = nullptr;
+  int64_t* d_ids = nullptr;
+  int64_t* d_next = nullptr;
+  float2* rope = nullptr;  // [max_seq][hd/2] (cos, sin)
+  void* attn_scratch = nullptr;
+  float* am_val = nullptr;
+  int64_t* am_idx = nullptr;
+  int* d_err = nullptr;
+  void* abuf = nullptr;
+
+  cudaStream_t cap = nullptr;
+  bool use_graphs = true;
+  std::map<int, cudaGraphExec_t> graphs;
+  KTiming* tm = nullptr;  // set while capturing an instrumented step
+  std::map<int, KTiming*> timed;
+};
+
+namespace {
+
+struct DeviceGuard {
+  int prev = -1;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+    cudaSetDevice(dev);
+  }
+  ~DeviceGuard() {
+    if (prev >= 0) cudaSetDevice(prev);
+  }
+};
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Begin / end of one kernel-class instance (no-ops unless an instrumented
+// step is being captured).
+void tbeg(q2_model* M, int cls, cudaStream_t st) {
+  KTiming* t = M->tm;
+  if (!t) return;
+  while (t->ev.size() < 2 * t->used + 2) {
+    cudaEvent_t e;
+    cudaEventCreate(&e);
+    t->ev.push_back(e);
+  }
+  t->cls.resize(t->used + 1);
+  t->cls[t->used] = cls;
+  cudaEventRecordWithFlags(t->ev[2 * t->used], st, cudaEventRecordExternal);
+}
+void tend(q2_model* M, cudaStream_t st) {
+  KTiming* t = M->tm;
+  if (!t) return;
+  cudaEventRecordWithFlags(t->ev[2 * t->used + 1], st, cudaEventRecordExternal);
+  t->used++;
+}
+#define TIMED(cls, expr)         \
+  do {                           \
+    tbeg(M, (cls), st);          \
+    q2_status _ts = (expr);      \
+    if (_ts != Q2_OK) return _ts; \
+    tend(M, st);                 \
+  } while (0)
+
+// -------------------------------------------------- RoPE + KV write-back
+// One thread per (token, head, pair j) over the nh q heads, nkv k heads and
+// nkv v heads of the fused qkv row.  q is rotated in place; k is rotated and
+// written to the cache; v is copied to the cache.  Decode: token t is the
+// next position of sequence t.  Prefill: token t is position pos0 + t of
+// sequence `seq`.
+template <typename T>
+__global__ void rope_kv_kernel(T* qkv, int qkvd, int T_, int nh, int nkv, int hd, const float2* rope,
+                               T* kc, T* vc, long long kv_seq_stride, int max_seq, const int* lens,
+                               int decode, int seq, int pos0) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int half = hd >> 1;
+  const int heads = nh + 2 * nkv;
+  const long long total = (long long)T_ * heads * half;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int j = (int)(i % half);
+    const int hh = (int)((i / half) % heads);
+    const int t = (int)(i / ((long long)half * heads));
+    const int sq = decode ? t : seq;
+    const int pos = decode ? lens[t] : pos0 + t;
+    T* row = qkv + (size_t)t * qkvd + (size_t)hh * hd;
+    const float a = to_f(row[j]), b = to_f(row[j + half]);
+    if (hh < nh + nkv) {
+      const float2 cs = rope[(size_t)pos * half + j];
+      const T ra = from_f<T>(a * cs.x - b * cs.y);
+      const T rb = from_f<T>(b * cs.x + a * cs.y);
+      if (hh < nh) {
+        row[j] = ra;
+        row[j + half] = rb;
+      } else {
+        T* dst = kc + (size_t)sq * kv_seq_stride + ((size_t)(hh - nh) * max_seq + pos) * hd;
+        dst[j] = ra;
+        dst[j + half] = rb;
+      }
+    } else {
+      T* dst = vc + (size_t)sq * kv_seq_stride + ((size_t)(hh - nh - nkv) * max_seq + pos) * hd;
+      dst[j] = row[j];
+      dst[j + half] = row[j + half];
+    }
+  }
+}
+
+__global__ void inc_lens_kernel(int* lens, int B) {
+  pdl_launch_dependents();
+  pdl_wait();
+  int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b < B) lens[b] += 1;
+}
+
+__global__ void set_len_kernel(int* lens, int seq, int v) {
+  pdl_wait();
+  lens[seq] = v;
+}
+
+q2_status launch_rope_kv(q2_model* M, int l, int T, const int* lens, int decode, int seq, int pos0,
+                         cudaStream_t st, bool pdl) {
+  const q2_meta& m = M->m;
+  long long work = (long long)T * (m.n_heads + 2 * m.n_kv_heads) * (m.head_dim / 2);
+  int blocks = (int)((work + 255) / 256);
+  if (blocks > num_sms() * 8) blocks = num_sms() * 8;
+  if (blocks < 1) blocks = 1;
+  size_t loff = (size_t)l * M->kv_layer_stride;
+  if (M->dt == Q2_F32)
+    Q2_LAUNCH(rope_kv_kernel<float>, dim3(blocks), dim3(256), 0, st, pdl, (float*)M->qkv, M->qkvd,
+              T, m.n_heads, m.n_kv_heads, m.head_dim, (const float2*)M->rope,
+              (float*)M->kc + loff, (float*)M->vc + loff, M->kv_seq_stride, m.max_seq, lens, decode,
+              seq, pos0);
+  else
+    Q2_LAUNCH(rope_kv_kernel<__nv_bfloat16>, dim3(blocks), dim3(256), 0, st, pdl,
+              (__nv_bfloat16*)M->qkv, M->qkvd, T, m.n_heads, m.n_kv_heads, m.head_dim,
+              (const float2*)M->rope, (__nv_bfloat16*)M->kc + loff, (__nv_bfloat16*)M->vc + loff,
+              M->kv_seq_stride, m.max_seq, lens, decode, seq, pos0);
+  return Q2_OK;
+}
+
+int decode_splits(const q2_model* M, int rows) {
+  return attn_splits(rows, M->m.n_kv_heads, M->m.max_seq);
+}
+
+// The decoder layers on x [T, H].  decode != 0: row t is the next token of
+// sequence t; else rows are positions pos0.. of sequence `seq`.  On return,
+// o holds the last layer's down-projection output (not yet added to x).
+q2_status run_layers(q2_model* M, int T, int decode, int seq, int pos0, cudaStream_t st, bool pdl) {
+  const q2_meta& m = M->m;
+  const int H = m.hidden, I = m.intermediate, dt = M->dt;
+  for (int l = 0; l < m.n_layers; ++l) {
+    const LayerW& w = M->layers[l];
+    if (l == 0)
+      TIMED(Q2_K_NORM, launch_add_rms_norm(M->x, nullptr, M->h, w.in_norm, T, H, m.eps, dt, st, pdl));
+    TIMED(Q2_K_QKV, launch_linear(M->qkv, M->h, w.wqkv, w.bqkv, T, M->qkvd, H, dt, dt, st, pdl));
+    TIMED(Q2_K_ROPE_KV, launch_rope_kv(M, l, T, M->d_len, decode, seq, pos0, st, pdl));
+
+    AttnRows a = {};
+    a.q = M->qkv;
+    a.q_row_stride = M->qkvd;
+    size_t loff = (size_t)l * M->kv_layer_stride * M->es;
+    a.k = (const char*)M->kc + loff;
+    a.v = (const char*)M->vc + loff;
+    a.kv_seq_stride = M->kv_seq_stride;
+    a.kv_tok_stride = m.head_dim;
+    a.kv_head_stride = (long long)m.max_seq * m.head_dim;
+    a.out = M->att;
+    a.out_row_stride = M->qd;
+    a.rows = T;
+    a.nh = m.n_heads;
+    a.nkv = m.n_kv_heads;
+    a.hd = m.head_dim;
+    a.scale = 1.0f / sqrtf((float)m.head_dim);
+    int nsplit;
+    if (decode) {
+      a.base = 1;
+      a.row_step = 0;
+      a.lens = M->d_len;
+      a.seq_is_row = 1;
+      a.fixed_seq = 0;
+      nsplit = decode_splits(M, T);
+    } else {
+      a.base = pos0 + 1;
+      a.row_step = 1;
+      a.lens = nullptr;
+      a.seq_is_row = 0;
+      a.fixed_seq = seq;
+      nsplit = attn_splits(T, m.n_kv_heads, pos0 + T);
+    }
+    TIMED(Q2_K_ATTN, launch_attention(a, nsplit, M->attn_scratch, dt, st, pdl));
+
+    TIMED(Q2_K_O, launch_linear(M->o, M->att, w.wo, nullptr, T, H, M->qd, dt, dt, st, pdl));
+    TIMED(Q2_K_NORM, launch_add_rms_norm(M->x, M->o, M->h, w.post_norm, T, H, m.eps, dt, st, pdl));
+    TIMED(Q2_K_GATE_UP, launch_linear(M->gu, M->h, w.wgu, nullptr, T, 2 * I, H, dt, dt, st, pdl));
+    TIMED(Q2_K_SWIGLU, launch_swiglu_rows(M->s, M->gu, T, I, dt, st, pdl));
+    TIMED(Q2_K_DOWN, launch_linear(M->o, M->s, w.wd, nullptr, T, H, I, dt, dt, st, pdl));
+    if (l + 1 < m.n_layers)
+      TIMED(Q2_K_NORM,
+            launch_add_rms_norm(M->x, M->o, M->h, M->layers[l + 1].in_norm, T, H, m.eps, dt, st, pdl));
+  }
+  return Q2_OK;
+}
+
+// Final residual add + RMSNorm of `rows` rows starting at row r0, lm_head
+// into logits rows lrow.., argmax into next rows lrow...
+q2_status run_head(q2_model* M, int r0, int rows, int lrow, cudaStream_t st, bool pdl) {
+  const q2_meta& m = M->m;
+  const int H = m.hidden, V = m.vocab, dt = M->dt;
+  char* x = (char*)M->x + (size_t)r0 * H * M->es;
+  char* o = (char*)M->o + (size_t)r0 * H * M->es;
+  char* h = (char*)M->h + (size_t)r0 * H * M->es;
+  TIMED(Q2_K_NORM, launch_add_rms_norm(x, o, h, M->final_norm, rows, H, m.eps, dt, st, pdl));
+  float* lg = M->logits + (size_t)lrow * V;
+  TIMED(Q2_K_LM_HEAD, launch_linear(lg, h, M->lm_head, nullptr, rows, V, H, dt, Q2_F32, st, pdl));
+  int parts = argmax_parts(rows, V);
+  TIMED(Q2_K_ARGMAX, launch_argmax(M->d_next + lrow, nullptr, lg, rows, V, Q2_F32, M->am_val,
+                                   M->am_idx, parts, st, pdl));
+  return Q2_OK;
+}
+
+q2_status decode_body(q2_model* M, int B, cudaStream_t st) {
+  const bool pdl = true;
+  const q2_meta& m = M->m;
+  TIMED(Q2_K_EMBED,
+        launch_embedding(M->x, M->d_ids, M->embed, B, m.vocab, m.hidden, M->dt, M->d_err, st, pdl));
+  Q2_TRY(run_layers(M, B, 1, 0, 0, st, pdl));
+  Q2_TRY(run_head(M, 0, B, 0, st, pdl));
+  tbeg(M, Q2_K_OTHER, st);
+  Q2_LAUNCH(inc_lens_kernel, dim3(1), dim3(64 * ((B + 63) / 64)), 0, st, pdl, M->d_len, B);
+  tend(M, st);
+  return Q2_OK;
+}
+
+q2_status check_stream_device(q2_model* M, cudaStream_t st) {
+  if (!st) return Q2_OK;
+  int dev = -1;
+  cudaError_t e = cudaStreamGetDevice(st, &dev);
+  if (e == cudaSuccess && dev != M->device) {
+    set_error("stream belongs to another device than the model");
+    return Q2_ERR_INVALID_ARG;
+  }
+  return Q2_OK;
+}
+
+q2_status check_decode_capacity(q2_model* M, int B) {
+  for (int b = 0; b < B; ++b)
+    if (M->h_len[b] >= M->m.max_seq) {
+      set_error("decode_step: a sequence is full (max_seq)");
+      return Q2_ERR_CAPACITY;
+    }
+  return Q2_OK;
+}
+
+// Runs one decode step on the ids already in d_ids: the captured graph for
+// this batch size (captured on first use), or eager launches.
+q2_status decode_launch(q2_model* M, int B, cudaStream_t st) {
+  if (M->use_graphs) {
+    auto it = M->graphs.find(B);
+    if (it == M->graphs.end()) {
+      cudaGraph_t graph = nullptr;
+      Q2_CUDA_TRY(cudaStreamBeginCapture(M->cap, cudaStreamCaptureModeThreadLocal));
+      q2_status s = decode_body(M, B, M->cap);
+      cudaError_t e = cudaStreamEndCapture(M->cap, &graph);
+      if (s != Q2_OK) {
+        if (graph) cudaGraphDestroy(graph);
+        return s;
+      }
+      if (e != cudaSuccess) {
+        set_error(std::string("decode graph capture: ") + cudaGetErrorString(e));
+        return Q2_ERR_CUDA;
+      }
+      cudaGraphExec_t exec = nullptr;
+      e = cudaGraphInstantiate(&exec, graph, 0);
+      cudaGraphDestroy(graph);
+      if (e != cudaSuccess) {
+        set_error(std::string("decode graph instantiate: ") + cudaGetErrorString(e));
+        return Q2_ERR_CUDA;
+      }
+      it = M->graphs.emplace(B, exec).first;
+    }
+    Q2_CUDA_TRY(cudaGraphLaunch(it->second, st));
+  } else {
+    Q2_TRY(decode_body(M, B, st));
+  }
+  for (int b = 0; b < B; ++b) M->h_len[b] += 1;
+  return Q2_OK;
+}
+
+}  // namespace
+
+// ===================================================================== ABI
+extern "C" {
+
+q2_status q2_model_create(const q2_meta* meta, int device, q2_model** out) {
+  clear_error();
+  Q2_CHECK_ARG(meta && out, Q2_ERR_INVALID_ARG, "model_create: NULL argument");
+  const q2_meta& m = *meta;
+  Q2_CHECK_ARG(m.dtype == Q2_F32 || m.dtype == Q2_BF16, Q2_ERR_DTYPE, "model_create: bad dtype");
+  Q2_CHECK_ARG(m.n_layers > 0 && m.hidden > 0 && m.n_heads > 0 && m.n_kv_heads > 0 &&
+                   m.intermediate > 0 && m.vocab > 0 && m.max_seq > 0 && m.max_batch > 0 &&
+                   m.max_prefill_tokens >= 0,
+               Q2_ERR_SHAPE, "model_create: sizes must be positive");
+  Q2_CHECK_ARG(m.head_dim == 32 || m.head_dim == 64 || m.head_dim == 128, Q2_ERR_SHAPE,
+               "model_create: head_dim must be 32, 64 or 128");
+  Q2_CHECK_ARG(m.n_heads % m.n_kv_heads == 0 && m.n_heads / m.n_kv_heads <= 8, Q2_ERR_SHAPE,
+               "model_create: need n_heads % n_kv_heads == 0 and a group of at most 8");
+  Q2_CHECK_ARG(m.hidden % 8 == 0 && m.intermediate % 8 == 0, Q2_ERR_SHAPE,
+               "model_create: hidden and intermediate must be multiples of 8");
+  Q2_CHECK_ARG(m.max_batch <= 1024 && m.max_seq <= (1 << 24), Q2_ERR_SHAPE,
+               "model_create: max_batch <= 1024 and max_seq <= 2^24");
+  int ndev = 0;
+  Q2_CUDA_TRY(cudaGetDeviceCount(&ndev));
+  Q2_CHECK_ARG(device >= 0 && device < ndev, Q2_ERR_INVALID_ARG, "model_create: no such device");
+  Q2_CUDA_TRY(cudaSetDevice(device));
+
+  q2_model* M = new q2_model();
+  M->m = m;
+  M->device = device;
+  M->dt = m.dtype;
+  M->es = dtype_size(m.dtype);
+  M->qd = m.n_heads * m.head_dim;
+  M->kd = m.n_kv_heads * m.head_dim;
+  M->qkvd = M->qd + 2 * M->kd;
+  M->chunk = m.max_prefill_tokens > 0 ? m.max_prefill_tokens : 4096;
+  M->tmax = M->chunk > m.max_batch ? M->chunk : m.max_batch;
+  M->h_len.assign(m.max_batch, 0);
+  M->layers.resize(m.n_layers);
+
+  auto fail = [&](q2_status s) {
+    q2_model_destroy(M);
+    return s;
+  };
+
+  // ---- weights: one allocation, 256-byte aligned pieces
+  const size_t es = M->es, H = m.hidden, I = m.intermediate, V = m.vocab;
+  std::vector<std::pair<void**, size_t>> wl;
+  wl.push_back({&M->embed, V * H * es});
+  wl.push_back({&M->lm_head, V * H * es});
+  wl.push_back({&M->final_norm, H * es});
+  for (auto& L : M->layers) {
+    wl.push_back({&L.in_norm, H * es});
+    wl.push_back({&L.wqkv, (size_t)M->qkvd * H * es});
+    wl.push_back({&L.bqkv, (size_t)M->qkvd * es});
+    wl.push_back({&L.wo, H * M->qd * es});
+    wl.push_back({&L.post_norm, H * es});
+    wl.push_back({&L.wgu, 2 * I * H * es});
+    wl.push_back({&L.wd, H * I * es});
+  }
+  size_t wbytes = 0;
+  for (auto& p : wl) wbytes += align_up(p.second, 256);
+  if (cudaMalloc(&M->wbuf, wbytes) != cudaSuccess) {
+    set_error("model_create: cannot allocate weights");
+    return fail(Q2_ERR_OOM);
+  }
+  cudaMemset(M->wbuf, 0, wbytes);
+  {
+    char* p = (char*)M->wbuf;
+    for (auto& q : wl) {
+      *q.first = p;
+      p += align_up(q.second, 256);
+    }
+  }
+
+  // ---- KV cache
+  M->kv_seq_stride = (long long)m.n_kv_heads * m.max_seq * m.head_dim;
+  M->kv_layer_stride = M->kv_seq_stride * m.max_batch;
+  size_t kvbytes = (size_t)M->kv_layer_stride * m.n_layers * es;
+  if (cudaMalloc(&M->kc, kvbytes) != cudaSuccess || cudaMalloc(&M->vc, kvbytes) != cudaSuccess) {
+    set_error("model_create: cannot allocate the KV cache");
+    return fail(Q2_ERR_OOM);
+  }
+  cudaMemset(M->kc, 0, kvbytes);
+  cudaMemset(M->vc, 0, kvbytes);
+
+  // ---- activations and scratch
+  size_t T = M->tmax;
+  size_t scratch = 0;
+  for (int r = 1; r <= M->tmax; ++r) {
+    size_t b = attn_scratch_bytes(r, m.n_heads, m.head_dim, attn_splits(r, m.n_kv_heads, m.max_seq));
+    if (b > scratch) scratch = b;
+  }
+  size_t am = 0;
+  for (int r = 1; r <= m.max_batch; ++r) {
+    size_t b = (size_t)r * argmax_parts(r, V);
+    if (b > am) am = b;
+  }
+  std::vector<std::pair<void**, size_t>> al;
+  al.push_back({&M->x, T * H * es});
+  al.push_back({&M->h, T * H * es});
+  al.push_back({&M->qkv, T * M->qkvd * es});
+  al.push_back({&M->att, T * M->qd * es});
+  al.push_back({&M->o, T * H * es});
+  al.push_back({&M->gu, T * 2 * I * es});
+  al.push_back({&M->s, T * I * es});
+  al.push_back({(void**)&M->logits, (size_t)m.max_batch * V * sizeof(float)});
+  al.push_back({(void**)&M->d_ids, T * sizeof(int64_t)});
+  al.push_back({(void**)&M->d_next, (size_t)m.max_batch * sizeof(int64_t)});
+  al.push_back({(void**)&M->rope, (size_t)m.max_seq * (m.head_dim / 2) * sizeof(float2)});
+  al.push_back({&M->attn_scratch, scratch});
+  al.push_back({(void**)&M->am_val, am * sizeof(float)});
+  al.push_back({(void**)&M->am_idx, am * sizeof(int64_t)});
+  al.push_back({(void**)&M->d_len, (size_t)m.max_batch * sizeof(int)});
+  al.push_back({(void**)&M->d_err, sizeof(int)});
+  size_t abytes = 0;
+  for (auto& p : al) abytes += align_up(p.second ? p.second : 1, 256);
+  if (cudaMalloc(&M->abuf, abytes) != cudaSuccess) {
+    set_error("model_create: cannot allocate activation buffers");
+    return fail(Q2_ERR_OOM);
+  }
+  cudaMemset(M->abuf, 0, abytes);
+  {
+    char* p = (char*)M->abuf;
+    for (auto& q : al) {
+      *q.first = p;
+      p += align_up(q.second ? q.second : 1, 256);
+    }
+  }
+  if (!scratch) M->attn_scratch = nullptr;
+
+  // ---- RoPE table: angle pos * theta^(-2j/hd) and its cos/sin in double,
+  // stored as fp32 pairs.
+  {
+    const int half = m.head_dim / 2;
+    std::vector<float2> tab((size_t)m.max_seq * half);
+    for (int j = 0; j < half; ++j) {
+      double inv = pow((double)m.theta, -(2.0 * j) / (double)m.head_dim);
+      for (int p = 0; p < m.max_seq; ++p) {
+        double a = (double)p * inv;
+        tab[(size_t)p * half + j] = make_float2((float)cos(a), (float)sin(a));
+      }
+    }
+    if (cudaMemcpy(M->rope, tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice) !=
+        cudaSuccess) {
+      set_error("model_create: cannot upload the RoPE table");
+      return fail(Q2_ERR_CUDA);
+    }
+  }
+  if (cudaStreamCreateWithFlags(&M->cap, cudaStreamNonBlocking) != cudaSuccess) {
+    set_error("model_create: cannot create a stream");
+    return fail(Q2_ERR_CUDA);
+  }
+  if (cudaDeviceSynchronize() != cudaSuccess) {
+    set_error(std::string("model_create: ") + cudaGetErrorString(cudaGetLastError()));
+    return fail(Q2_ERR_CUDA);
+  }
+  *out = M;
+  return Q2_OK;
+}
+
+q2_status q2_model_destroy(q2_model* M) {
+  clear_error();
+  if (!M) return Q2_OK;
+  DeviceGuard g(M->device);
+  for (auto& kv : M->graphs) cudaGraphExecDestroy(kv.second);
+  M->graphs.clear();
+  for (auto& kv : M->timed) {
+    if (kv.second->exec) cudaGraphExecDestroy(kv.second->exec);
+    for (cudaEvent_t e : kv.second->ev) cudaEventDestroy(e);
+    delete kv.second;
+  }
+  M->timed.clear();
+  if (M->cap) cudaStreamDestroy(M->cap);
+  cudaFree(M->wbuf);
+  cudaFree(M->kc);
+  cudaFree(M->vc);
+  cudaFree(M->abuf);
+  delete M;
+  return Q2_OK;
+}
+
+q2_status q2_model_load_weight(q2_model* M, int kind, int layer, const void* src, size_t nbytes,
+                               void* stream) {
+  clear_error();
+  Q2_CHECK_ARG(M && src, Q2_ERR_INVALID_ARG, "load_weight: NULL argument");
+  const q2_meta& m = M->m;
+  const size_t es = M->es, H = m.hidden, I = m.intermediate, V = m.vocab;
+  bool per_layer = kind >= Q2_W_IN_NORM && kind <= Q2_W_DOWN;
+  Q2_CHECK_ARG(kind >= Q2_W_EMBED && kind <= Q2_W_DOWN, Q2_ERR_INVALID_ARG, "load_weight: bad kind");
+  Q2_CHECK_ARG(!per_layer || (layer >= 0 && layer < m.n_layers), Q2_ERR_INVALID_ARG,
+               "load_weight: bad layer");
+  LayerW* L = per_layer ? &M->layers[layer] : nullptr;
+  char* dst = nullptr;
+  size_t want = 0;
+  switch (kind) {
+    case Q2_W_EMBED: dst = (char*)M->embed; want = V * H; break;
+    case Q2_W_LM_HEAD: dst = (char*)M->lm_head; want = V * H; break;
+    case Q2_W_FINAL_NORM: dst = (char*)M->final_norm; want = H; break;
+    case Q2_W_IN_NORM: dst = (char*)L->in_norm; want = H; break;
+    case Q2_W_Q: dst = (char*)L->wqkv; want = (size_t)M->qd * H; break;
+    case Q2_W_K: dst = (char*)L->wqkv + (size_t)M->qd * H * es; want = (size_t)M->kd * H; break;
+    case Q2_W_V: dst = (char*)L->wqkv + (size_t)(M->qd + M->kd) * H * es; want = (size_t)M->kd * H; break;
+    case Q2_W_Q_BIAS: dst = (char*)L->bqkv; want = M->qd; break;
+    case Q2_W_K_BIAS: dst = (char*)L->bqkv + (size_t)M->qd * es; want = M->kd; break;
+    case Q2_W_V_BIAS: dst = (char*)L->bqkv + (size_t)(M->qd + M->kd) * es; want = M->kd; break;
+    case Q2_W_O: dst = (char*)L->wo; want = H * M->qd; break;
+    case Q2_W_POST_NORM: dst = (char*)L->post_norm; want = H; break;
+    case Q2_W_GATE: dst = (char*)L->wgu; want = I * H; break;
+    case Q2_W_UP: dst = (char*)L->wgu + I * H * es; want = I * H; break;
+    case Q2_W_DOWN: dst = (char*)L->wd; want = H * I; break;
+  }
+  Q2_CHECK_ARG(nbytes == want * es, Q2_ERR_SHAPE, "load_weight: nbytes does not match the tensor size");
+  DeviceGuard g(M->device);
+  cudaStream_t st = as_stream(stream);
+  Q2_TRY(check_stream_device(M, st));
+  Q2_CUDA_TRY(cudaMemcpyAsync(dst, src, nbytes, cudaMemcpyDeviceToDevice, st));
+  return Q2_OK;
+}
+
+q2_status q2_model_decode_step(q2_model* M, const int64_t* ids, int B, int64_t* next, float* logits,
+                               void* stream) {
+  clear_error();
+  Q2_CHECK_ARG(M && ids && next, Q2_ERR_INVALID_ARG, "decode_step: NULL argument");
+  Q2_CHECK_ARG(B >= 1 && B <= M->m.max_batch, Q2_ERR_CAPACITY, "decode_step: batch outside [1, max_batch]");
+  DeviceGuard g(M->device);
+  cudaStream_t st = as_stream(stream);
+  Q2_TRY(check_stream_device(M, st));
+  Q2_TRY(check_decode_capacity(M, B));
+  Q2_CUDA_TRY(cudaMemcpyAsync(M->d_ids, ids, B * sizeof(int64_t), cudaMemcpyDeviceToDevice, st));
+  Q2_TRY(decode_launch(M, B, st));
+  Q2_CUDA_TRY(cudaMemcpyAsync(next, M->d_next, B * sizeof(int64_t), cudaMemcpyDeviceToDevice, st));
+  if (logits)
+    Q2_CUDA_TRY(cudaMemcpyAsync(logits, M->logits, (size_t)B * M->m.vocab * sizeof(float),
+                                cudaMemcpyDeviceToDevice, st));
+  return Q2_OK;
+}
+
+q2_status q2_model_decode_step_host(q2_model* M, const int64_t* ids_host, int B, int64_t* next_host,
+                                    void* stream) {
+  clear_error();
+  Q2_CHECK_ARG(M && ids_host && next_host, Q2_ERR_INVALID_ARG, "decode_step_host: NULL argument");
+  Q2_CHECK_ARG(B >= 1 && B <= M->m.max_batch, Q2_ERR_CAPACITY, "decode_step_host: batch outside [1, max_batch]");
+  DeviceGuard g(M->device);
+  cudaStream_t st = as_stream(stream);
+  Q2_TRY(check_stream_device(M, st));
+  Q2_TRY(check_decode_capacity(M, B));
+  Q2_CUDA_TRY(cudaMemcpyAsync(M->d_ids, ids_host, B * sizeof(int64_t), cudaMemcpyHostToDevice, st));
+  Q2_TRY(decode_launch(M, B, st));
+  Q2_CUDA_TRY(cudaMemcpyAsync(next_host, M->d_next, B * sizeof(int64_t), cudaMemcpyDeviceToHost, st));
+  Q2_CUDA_TRY(cudaStreamSynchronize(st));
+  return Q2_OK;
+}
+
+q2_status q2_model_forward_hidden(q2_model* M, const void* x_in, int B, void* x_out, void* stream) {
+  clear_error();
+  Q2_CHECK_ARG(M && x_in && x_out, Q2_ERR_INVALID_ARG, "forward_hidden: NULL argument");
+  Q2_CHECK_ARG(B >= 1 && B <= M->m.max_batch, Q2_ERR_CAPACITY, "forward_hidden: batch outside [1, max_batch]");
+  for (int b = 0; b < B; ++b)
+    Q2_CHECK_ARG(M->h_len[b] < M->m.max_seq, Q2_ERR_CAPACITY, "forward_hidden: a sequence is full");
+  DeviceGuard g(M->device);
+  cudaStream_t st = as_stream(stream);
+  Q2_TRY(check_stream_device(M, st));
+  const size_t bytes = (size_t)B * M->m.hidden * M->es;
+  Q2_CUDA_TRY(cudaMemcpyAsync(M->x, x_in, bytes, cudaMemcpyDeviceToDevice, st));
+  Q2_TRY(run_layers(M, B, 1, 0, 0, st, false));
+  Q2_TRY(launch_add_rms_norm(M->x, M->o, nullptr, nullptr, B, M->m.hidden, M->m.eps, M->dt, st, false));
+  Q2_CUDA_TRY(cudaMemcpyAsync(x_out, M->x, bytes, cudaMemcpyDeviceToDevice, st));
+  Q2_LAUNCH(inc_lens_kernel, dim3(1), dim3(64 * ((B + 63) / 64)), 0, st, false, M->d_len, B);
+  for (int b = 0; b < B; ++b) M->h_len[b] += 1;
+  return Q2_OK;
+}
+
+q2_status q2_model_prefill(q2_model* M, const int64_t* ids, int batch, const int32_t* lens,
+                           int64_t* next, float* logits, void* stream) {
+  clear_error();
+  Q2_CHECK_ARG(M && ids && lens && next, Q2_ERR_INVALID_ARG, "prefill: NULL argument");
+  Q2_CHECK_ARG(batch >= 1 && batch <= M->m.max_batch, Q2_ERR_CAPACITY, "prefill: batch outside [1, max_batch]");
+  for (int b = 0; b < batch; ++b) {
+    Q2_CHECK_ARG(lens[b] >= 0, Q2_ERR_INVALID_ARG, "prefill: negative length");
+    Q2_CHECK_ARG((long long)M->h_len[b] + lens[b] <= M->m.max_seq, Q2_ERR_CAPACITY,
+                 "prefill: a sequence would pass max_seq");
+  }
+  DeviceGuard g(M->device);
+  cudaStream_t st = as_stream(stream);
+  Q2_TRY(check_stream_device(M, st));
+  const q2_meta& m = M->m;
+  const bool pdl = true;
+  size_t off = 0;
+  for (int b = 0; b < batch; ++b) {
+    const int n = lens[b];
+    for (int c = 0; c < n; c += M->chunk) {
+      const int T = n - c < M->chunk ? n - c : M->chunk;
+      const int pos0 = M->h_len[b];
+      Q2_CUDA_TRY(cudaMemcpyAsync(M->d_ids, ids + off + c, T * sizeof(int64_t), cudaMemcpyDeviceToDevice, st));
+      Q2_TRY(launch_embedding(M->x, M->d_ids, M->embed, T, m.vocab, m.hidden, M->dt, M->d_err, st, pdl));
+      Q2_TRY(run_layers(M, T, 0, b, pos0, st, pdl));
+      M->h_len[b] = pos0 + T;
+      Q2_LAUNCH(set_len_kernel, dim3(1), dim3(1), 0, st, pdl, M->d_len, b, pos0 + T);
+      if (c + T == n) {
+        Q2_TRY(run_head(M, T - 1, 1, b, st, pdl));
+        Q2_CUDA_TRY(cudaMemcpyAsync(next + b, M->d_next + b, sizeof(int64_t), cudaMemcpyDeviceToDevice, st));
+        if (logits)
+          Q2_CUDA_TRY(cudaMemcpyAsync(logits + (size_t)b * m.vocab, M->logits + (size_t)b * m.vocab,
+                                      (size_t)m.vocab * sizeof(float), cudaMemcpyDeviceToDevice, st));
+      }
+    }
+    off += n;
+  }
+  return Q2_OK;
+}
+
+q2_status q2_model_reset_kv(q2_model* M, int seq) {
+  clear_error();
+  Q2_CHECK_ARG(M, Q2_ERR_INVALID_ARG, "reset_kv: NULL model");
+  Q2_CHECK_ARG(seq >= -1 && seq < M->m.max_batch, Q2_ERR_INVALID_ARG, "reset_kv: bad sequence");
+  DeviceGuard g(M->device);
+  Q2_CUDA_TRY(cudaDeviceSynchronize());
+  if (seq == -1) {
+    std::fill(M->h_len.begin(), M->h_len.end(), 0);
+    Q2_CUDA_TRY(cudaMemset(M->d_len, 0, M->m.max_batch * sizeof(int)));
+  } else {
+    M->h_len[seq] = 0;
+    Q2_CUDA_TRY(cudaMemset(M->d_len + seq, 0, sizeof(int)));
+  }
+  return Q2_OK;
+}
+
+q2_status q2_model_set_seq_len(q2_model* M, int seq, int len) {
+  clear_error();
+  Q2_CHECK_ARG(M, Q2_ERR_INVALID_ARG, "set_seq_len: NULL model");
+  Q2_CHECK_ARG(seq >= 0 && seq < M->m.max_batch, Q2_ERR_INVALID_ARG, "set_seq_len: bad sequence");
+  Q2_CHECK_ARG(len >= 0 && len <= M->m.max_seq, Q2_ERR_CAPACITY, "set_seq_len: length outside [0, max_seq]");
+  DeviceGuard g(M->device);
+  Q2_CUDA_TRY(cudaDeviceSynchronize());
+  M->h_len[seq] = len;
+  Q2_CUDA_TRY(cudaMemcpy(M->d_len + seq, &len, sizeof(int), cudaMemcpyHostToDevice));
+  return Q2_OK;
+}
+
+q2_status q2_model_get_seq_len(const q2_model* M, int seq, int* len) {
+  clear_error();
+  Q2_CHECK_ARG(M && len, Q2_ERR_INVALID_ARG, "get_seq_len: NULL argument");
+  Q2_CHECK_ARG(seq >= 0 && seq < M->m.max_batch, Q2_ERR_INVALID_ARG, "get_seq_len: bad sequence");
+  *len = M->h_len[seq];
+  return Q2_OK;
+}
+
+q2_status q2_model_kv_cache(q2_model* M, int layer, int seq, void** k, void** v) {
+  clear_error();
+  Q2_CHECK_ARG(M && k && v, Q2_ERR_INVALID_ARG, "kv_cache: NULL argument");
+  Q2_CHECK_ARG(layer >= 0 && layer < M->m.n_layers && seq >= 0 && seq < M->m.max_batch,
+               Q2_ERR_INVALID_ARG, "kv_cache: bad layer or sequence");
+  size_t off = ((size_t)layer * M->kv_layer_stride + (size_t)seq * M->kv_seq_stride) * M->es;
+  *k = (char*)M->kc + off;
+  *v = (char*)M->vc + off;
+  return Q2_OK;
+}
+
+q2_status q2_model_check_error(q2_model* M, void* stream) {
+  clear_error();
+  Q2_CHECK_ARG(M, Q2_ERR_INVALID_ARG, "check_error: NULL model");
+  DeviceGuard g(M->device);
+  Q2_CUDA_TRY(cudaStreamSynchronize(as_stream(stream)));
+  int v = 0;
+  Q2_CUDA_TRY(cudaMemcpy(&v, M->d_err, sizeof v, cudaMemcpyDeviceToHost));
+  if (v) {
+    int zero = 0;
+    Q2_CUDA_TRY(cudaMemcpy(M->d_err, &zero, sizeof zero, cudaMemcpyHostToDevice));
+    set_error("a model kernel saw a token id outside [0, vocab)");
+    return Q2_ERR_INDEX;
+  }
+  return Q2_OK;
+}
+
+q2_status q2_model_set_graphs(q2_model* M, int enable) {
+  clear_error();
+  Q2_CHECK_ARG(M, Q2_ERR_INVALID_ARG, "set_graphs: NULL model");
+  M->use_graphs = enable != 0;
+  return Q2_OK;
+}
+
+q2_status q2_model_time_kernels(q2_model* M, const int64_t* ids, int B, int steps, float* mean_ms,
+                                int* per_step, int* kernels_per_step, void* stream) {
+  clear_error();
+  Q2_CHECK_ARG(M && ids && mean_ms && per_step && kernels_per_step, Q2_ERR_INVALID_ARG,
+               "time_kernels: NULL argument");
+  Q2_CHECK_ARG(B >= 1 && B <= M->m.max_batch, Q2_ERR_CAPACITY, "time_kernels: batch outside [1, max_batch]");
+  Q2_CHECK_ARG(steps >= 1, Q2_ERR_INVALID_ARG, "time_kernels: steps must be positive");
+  for (int b = 0; b < B; ++b)
+    Q2_CHECK_ARG(M->h_len[b] + steps <= M->m.max_seq, Q2_ERR_CAPACITY,
+                 "time_kernels: a sequence would pass max_seq");
+  DeviceGuard g(M->device);
+  cudaStream_t st = as_stream(stream);
+  Q2_TRY(check_stream_device(M, st));
+  KTiming* t = nullptr;
+  auto it = M->timed.find(B);
+  if (it == M->timed.end()) {
+    t = new KTiming();
+    M->tm = t;
+    cudaGraph_t graph = nullptr;
+    cudaError_t e = cudaStreamBeginCapture(M->cap, cudaStreamCaptureModeThreadLocal);
+    q2_status s = e == cudaSuccess ? decode_body(M, B, M->cap) : Q2_ERR_CUDA;
+    if (e == cudaSuccess) e = cudaStreamEndCapture(M->cap, &graph);
+    M->tm = nullptr;
+    if (s == Q2_OK && e == cudaSuccess) {
+      size_t n = 0;
+      cudaGraphGetNodes(graph, nullptr, &n);
+      std::vector<cudaGraphNode_t> nodes(n);
+      cudaGraphGetNodes(graph, nodes.data(), &n);
+      for (auto nd : nodes) {
+        cudaGraphNodeType ty;
+        if (cudaGraphNodeGetType(nd, &ty) == cudaSuccess && ty == cudaGraphNodeTypeKernel) t->kernels++;
+      }
+      e = cudaGraphInstantiate(&t->exec, graph, 0);
+    }
+    if (graph) cudaGraphDestroy(graph);
+    if (s != Q2_OK || e != cudaSuccess) {
+      for (cudaEvent_t ev : t->ev) cudaEventDestroy(ev);
+      delete t;
+      if (s == Q2_OK) set_error(std::string("time_kernels: capture: ") + cudaGetErrorString(e));
+      return s != Q2_OK ? s : Q2_ERR_CUDA;
+    }
+    M->timed[B] = t;
+  } else {
+    t = it->second;
+  }
+  std::vector<int> saved(M->h_len.begin(), M->h_len.begin() + B);
+  std::vector<double> sum(Q2_K_COUNT, 0.0);
+  std::vector<int> cnt(Q2_K_COUNT, 0);
+  for (size_t i = 0; i < t->used; ++i) cnt[t->cls[i]]++;
+  Q2_CUDA_TRY(cudaMemcpyAsync(M->d_ids, ids, B * sizeof(int64_t), cudaMemcpyDeviceToDevice, st));
+  for (int r = 0; r < steps; ++r) {
+    Q2_CUDA_TRY(cudaGraphLaunch(t->exec, st));
+    Q2_CUDA_TRY(cudaStreamSynchronize(st));
+    for (size_t i = 0; i < t->used; ++i) {
+      float ms = 0.f;
+      Q2_CUDA_TRY(cudaEventElapsedTime(&ms, t->ev[2 * i], t->ev[2 * i + 1]));
+      sum[t->cls[i]] += ms;
+    }
+  }
+  Q2_CUDA_TRY(cudaMemcpy(M->d_len, saved.data(), B * sizeof(int), cudaMemcpyHostToDevice));
+  for (int c = 0; c < Q2_K_COUNT; ++c) {
+    per_step[c] = cnt[c];
+    mean_ms[c] = cnt[c] ? (float)(sum[c] / ((double)cnt[c] * steps)) : 0.f;
+  }
+  *kernels_per_step = t->kernels;
+  return Q2_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,258 @@
+"""Model-level parity: the CUDA decoder (prefill + greedy decode steps,
+through the C ABI) against the CPU oracle on the same seeded weights and
+inputs, plus GPU self-consistency and error paths.  GPU only."""
+
+import dataclasses
+
+import pytest
+import torch
+
+import oracle
+import qwen2_decode_step_b200 as q2
+import synth
+from tol import assert_bf16_logits, assert_close, assert_op_close, bits_equal
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _gpu(cuda_ok):
+    yield
+    torch.cuda.synchronize()
+
+
+def layer_weights(shape, seed, device="cpu"):
+    """All weights except the two [vocab, hidden] tables."""
+    return {k: synth.weight(shape, k[0], k[1], seed, device) for k in shape.weight_shapes()
+            if k[0] not in ("embed", "lm_head")}
+
+
+def pair(shape, w, max_seq, max_batch=1, **kw):
+    om = oracle.OracleModel(shape, max_seq=max_seq, max_batch=max_batch)
+    om.load(w)
+    gm = q2.Model(shape, max_seq=max_seq, max_batch=max_batch, **kw)
+    gm.load(w)
+    return om, gm
+
+
+# ------------------------------------------------------------ tiny fp32
+
+TINY = synth.WORKLOADS["tiny-2l-f32-prompt16-decode16"]
+
+
+@pytest.fixture(scope="module")
+def tiny_w():
+    return synth.model_weights(TINY["shape"], TINY["seed"])
+
+
+def gpu_generate(gm, prompt, n_decode, teacher=None):
+    nxt, lg = gm.prefill(prompt.cuda(), [prompt.numel()], want_logits=True)
+    toks, logits = [int(nxt[0])], [lg[0].cpu()]
+    for i in range(n_decode):
+        feed = nxt if teacher is None else torch.tensor([teacher[i]], device="cuda")
+        nxt, lg = gm.decode_step(feed, want_logits=True)
+        toks.append(int(nxt[0]))
+        logits.append(lg[0].cpu())
+    return toks, logits
+
+
+def test_tiny_f32_greedy_untethered(tiny_w):
+    shape = TINY["shape"]
+    prompt = synth.prompt_ids(shape, TINY["prompt"], TINY["seed"])
+    om, gm = pair(shape, tiny_w, max_seq=64)
+    ref_toks, ref_logits = om.generate(0, prompt, TINY["decode"])
+    toks, logits = gpu_generate(gm, prompt, TINY["decode"])
+    assert toks == ref_toks
+    for i, (a, b) in enumerate(zip(logits, ref_logits)):
+        assert_close(a, b, 1e-4, f"logits step {i}")
+    gm.check_error()
+
+
+def test_tiny_f32_chunked_prefill_and_eager_match(tiny_w):
+    shape = TINY["shape"]
+    prompt = synth.prompt_ids(shape, TINY["prompt"], TINY["seed"])
+    om, gm = pair(shape, tiny_w, max_seq=64, max_prefill_tokens=5)  # chunks 5+5+5+1
+    ref_toks, ref_logits = om.generate(0, prompt, 4)
+    gm.set_graphs(False)
+    toks, logits = gpu_generate(gm, prompt, 4)
+    assert toks == ref_toks
+    for a, b in zip(logits, ref_logits):
+        assert_close(a, b, 1e-4, "chunked/eager logits")
+
+
+def test_tiny_f32_batched_decode_matches_each_sequence_alone(tiny_w):
+    shape = TINY["shape"]
+    lens = [5, 16, 9]
+    prompts = [synth.prompt_ids(shape, n, TINY["seed"], seq=b) for b, n in enumerate(lens)]
+    _, gm = pair(shape, tiny_w, max_seq=64, max_batch=3)
+    nxt = gm.prefill(torch.cat(prompts).cuda(), lens)
+    got = [[int(t)] for t in nxt.cpu()]
+    for _ in range(8):
+        nxt = gm.decode_step(nxt)
+        for b, t in enumerate(nxt.cpu().tolist()):
+            got[b].append(t)
+    for b in range(3):
+        om = oracle.OracleModel(shape, max_seq=64)
+        om.load(tiny_w)
+        ref, _ = om.generate(0, prompts[b], 8)
+        assert got[b] == ref, b
+        assert gm.get_seq_len(b) == lens[b] + 8
+
+
+# ------------------------------------------- one Qwen2-1.5B layer, decode
+
+def test_one_layer_decode_at_4096_context():
+    wl = synth.WORKLOADS["qwen2-1.5b-layer-decode-ctx4096"]
+    shape, seed, past = wl["shape"], wl["seed"], wl["past"]
+    w = layer_weights(shape, seed)
+    om, gm = pair(shape, w, max_seq=past + 1)
+    k, v = synth.kv_fill(shape, past, seed, layer=0, seq=0)
+    ok, ov = om.kv(0, 0)
+    ok[:past] = k
+    ov[:past] = v
+    om.set_len(0, past)
+    gk, gv = gm.kv_cache(0, 0)
+    gk[:, :past] = k.permute(1, 0, 2).cuda()
+    gv[:, :past] = v.permute(1, 0, 2).cuda()
+    gm.set_seq_len(0, past)
+    x = synth.hidden_input(shape, 1, seed)
+    ref = om.forward_hidden(0, x)
+    got = gm.forward_hidden(x.cuda())
+    assert_op_close(got, ref, "layer output")
+    # the appended K/V row (k after RoPE) at position 4095
+    assert_op_close(gk[:, past].cpu(), ok[past], "k appended")
+    assert_op_close(gv[:, past].cpu(), ov[past], "v appended")
+    assert gm.get_seq_len(0) == past + 1
+
+
+# --------------------------------------------- full Qwen2-1.5B shape, bf16
+
+@pytest.fixture(scope="module")
+def full_w():
+    shape = synth.QWEN2_1P5B
+    seed = synth.WORKLOADS["qwen2-1.5b-b1-prompt512-decode128"]["seed"]
+    w = synth.model_weights(shape, seed, device="cuda")  # drawn on the GPU (fast) ...
+    return {k: t.cpu() for k, t in w.items()}           # ... same bits on both sides
+
+
+def test_full_model_teacher_forced_logits(full_w):
+    shape = synth.QWEN2_1P5B
+    prompt = synth.prompt_ids(shape, 6, 2003)
+    om, gm = pair(shape, full_w, max_seq=64)
+    ref_toks, ref_logits = om.generate(0, prompt, 3)
+    toks, logits = gpu_generate(gm, prompt, 3, teacher=ref_toks)
+    for i, (a, b) in enumerate(zip(logits, ref_logits)):
+        assert_bf16_logits(a, b, f"step {i}")
+    agree = sum(int(a == b) for a, b in zip(toks, ref_toks))
+    assert agree >= len(toks) - 1, (toks, ref_toks)
+
+
+def test_full_model_batched_decode_rows_match_oracle(full_w):
+    """Batch of 4 sequences with different lengths; rows 0 and 3 against the oracle."""
+    shape = synth.QWEN2_1P5B
+    lens = [4, 7, 3, 5]
+    prompts = [synth.prompt_ids(shape, n, 2004, seq=b) for b, n in enumerate(lens)]
+    gm = q2.Model(shape, max_seq=32, max_batch=4)
+    gm.load(full_w)
+    nxt, lg = gm.prefill(torch.cat(prompts).cuda(), lens, want_logits=True)
+    for b in (0, 3):
+        om = oracle.OracleModel(shape, max_seq=32)
+        om.load(full_w)
+        t, l0 = om.forward(0, prompts[b])
+        assert_bf16_logits(lg[b].cpu(), l0, f"prefill row {b}")
+        feed = torch.tensor([t])
+        _, l1 = om.forward(0, feed)
+        ids = nxt.clone()
+        ids[b] = t
+        n2, lg2 = gm.decode_step(ids, want_logits=True)
+        assert_bf16_logits(lg2[b].cpu(), l1, f"decode row {b}")
+        for s in range(4):  # rewind all rows for the next sampled sequence
+            gm.set_seq_len(s, lens[s])
+
+
+# ------------------------------------------------- GPU self-consistency
+
+@pytest.fixture(scope="module")
+def mid():
+    shape = dataclasses.replace(synth.QWEN2_1P5B, n_layers=4, vocab=32000)
+    return shape, synth.model_weights(shape, 77, device="cuda")
+
+
+def test_prefill_plus_decode_equals_longer_prefill(mid):
+    shape, w = mid
+    gm = q2.Model(shape, max_seq=128)
+    gm.load(w)
+    prompt = synth.prompt_ids(shape, 40, 5).cuda()
+    n1 = gm.prefill(prompt, [40])
+    _, la = gm.decode_step(n1, want_logits=True)
+    gm.reset_kv()
+    _, lb = gm.prefill(torch.cat([prompt, n1]), [41], want_logits=True)
+    assert_bf16_logits(la[0].cpu(), lb[0].cpu(), "S+1 vs S+decode")
+
+
+def test_reset_and_rerun_is_bit_identical_and_graphs_match_eager(mid):
+    shape, w = mid
+    gm = q2.Model(shape, max_seq=128, max_batch=2)
+    gm.load(w)
+    prompt = synth.prompt_ids(shape, 30, 6).cuda()
+
+    def run(graphs):
+        gm.reset_kv()
+        gm.set_graphs(graphs)
+        nxt = gm.prefill(torch.cat([prompt, prompt]), [30, 30])
+        outs = []
+        for _ in range(5):
+            nxt, lg = gm.decode_step(nxt, want_logits=True)
+            outs.append(lg.clone())
+        return outs
+
+    a, b, c = run(True), run(True), run(False)
+    for x, y, z in zip(a, b, c):
+        assert bits_equal(x, y) and bits_equal(x, z)
+        assert bits_equal(x[0], x[1])  # identical sequences in one batch
+
+
+# ---------------------------------------------------------- error paths
+
+def test_capacity_and_index_errors(tiny_w):
+    shape = TINY["shape"]
+    gm = q2.Model(shape, max_seq=8)
+    gm.load(tiny_w)
+    with pytest.raises(q2.Q2Error) as e:
+        gm.prefill(synth.prompt_ids(shape, 9, 1).cuda(), [9])
+    assert e.value.status == "Q2_ERR_CAPACITY"
+    nxt = gm.prefill(synth.prompt_ids(shape, 8, 1).cuda(), [8])
+    with pytest.raises(q2.Q2Error) as e:
+        gm.decode_step(nxt)
+    assert e.value.status == "Q2_ERR_CAPACITY"
+    gm.reset_kv()
+    gm.decode_step(torch.tensor([shape.vocab + 5], device="cuda"))
+    with pytest.raises(q2.Q2Error) as e:
+        gm.check_error()
+    assert e.value.status == "Q2_ERR_INDEX"
+    gm.check_error()  # cleared
+    with pytest.raises(q2.Q2Error) as e:
+        gm.decode_step(torch.zeros(2, dtype=torch.int64, device="cuda"))  # batch > max_batch
+    assert e.value.status == "Q2_ERR_CAPACITY"
+
+
+def test_decode_step_host_matches_device_path(tiny_w):
+    shape = TINY["shape"]
+    prompt = synth.prompt_ids(shape, 10, 3)
+    _, gm = pair(shape, tiny_w, max_seq=64)
+    nxt = gm.prefill(prompt.cuda(), [10])
+    ids_h = torch.empty(1, dtype=torch.int64).pin_memory()
+    out_h = torch.empty(1, dtype=torch.int64).pin_memory()
+    ids_h[0] = int(nxt[0])
+    dev = []
+    host = []
+    gm2 = q2.Model(shape, max_seq=64)
+    gm2.load(tiny_w)
+    n2 = gm2.prefill(prompt.cuda(), [10])
+    for _ in range(5):
+        gm.decode_step_host(ids_h, out_h)
+        host.append(int(out_h[0]))
+        ids_h[0] = out_h[0]
+        n2 = gm2.decode_step(n2)
+        dev.append(int(n2[0]))
+    assert host == dev
