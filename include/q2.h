@@ -233,6 +233,23 @@ q2_status q2_model_decode_step_host(q2_model* model, const int64_t* ids_host, in
 q2_status q2_model_forward_hidden(q2_model* model, const void* x_in, int batch, void* x_out,
                                   void* stream);
 
+/* The decoder layers alone over T positions of sequence `seq` (a prefill
+ * on hidden states): x_in [T, H] (device, dtype) is the input of layer 0 at
+ * positions len .. len+T-1; x_out [T, H] receives the residual stream after
+ * the last layer.  Appends K/V and advances the length like q2_model_prefill
+ * (chunked by max_prefill_tokens).  With forward_hidden and q2_model_head it
+ * lets a caller feed every layer a given input (layer-wise teacher forcing,
+ * the per-layer bisection of the Day-0 adaptation tutorial, step 6). */
+q2_status q2_model_prefill_hidden(q2_model* model, int seq, const void* x_in, int T, void* x_out,
+                                  void* stream);
+
+/* The model's head on given hidden states: x [rows, H] (device, dtype,
+ * rows <= max_batch) -> final RMSNorm -> lm_head -> fp32 logits [rows, V]
+ * (device, may be NULL) and greedy next [rows] (device, int64).  No KV or
+ * length change. */
+q2_status q2_model_head(q2_model* model, const void* x, int rows, int64_t* next, float* logits,
+                        void* stream);
+
 /* Resets sequence `seq` (or every sequence when seq == -1) to length 0. */
 q2_status q2_model_reset_kv(q2_model* model, int seq);
 

@@ -78,6 +78,8 @@ _SIGS = {
     "q2_model_check_error": [_VP, _VP],
     "q2_model_set_graphs": [_VP, _I],
     "q2_model_time_kernels": [_VP, _VP, _I, _I, _VP, _VP, ctypes.POINTER(_I), _VP],
+    "q2_model_prefill_hidden": [_VP, _I, _VP, _I, _VP, _VP],
+    "q2_model_head": [_VP, _VP, _I, _VP, _VP, _VP],
 }
 
 KCLASS = ["embed", "norm", "qkv", "rope_kv", "attn", "o", "gate_up", "swiglu", "down", "lm_head",
@@ -312,6 +314,22 @@ class Model:
         out = torch.empty_like(x)
         _call("q2_model_forward_hidden", self._h, _p(x), x.shape[0], _p(out), _stream())
         return out
+
+    def prefill_hidden(self, seq: int, x: torch.Tensor) -> torch.Tensor:
+        """Decoder layers over x [T, H] at the next T positions of `seq`."""
+        _dense(x)
+        out = torch.empty_like(x)
+        _call("q2_model_prefill_hidden", self._h, seq, _p(x), x.shape[0], _p(out), _stream())
+        return out
+
+    def head(self, x: torch.Tensor):
+        """Final RMSNorm + lm_head + argmax on hidden states x [rows, H]: (next, fp32 logits)."""
+        _dense(x)
+        rows = x.shape[0]
+        nxt = torch.empty(rows, dtype=torch.int64, device=x.device)
+        lg = torch.empty((rows, self.shape.vocab), dtype=torch.float32, device=x.device)
+        _call("q2_model_head", self._h, _p(x), rows, _p(nxt), _p(lg), _stream())
+        return nxt, lg
 
     def reset_kv(self, seq: int = -1):
         _call("q2_model_reset_kv", self._h, seq)

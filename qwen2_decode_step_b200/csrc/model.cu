@@ -262,11 +262,12 @@ q2_status run_layers(q2_model* M, int T, int decode, int seq, int pos0, cudaStre
 
 // Final residual add + RMSNorm of `rows` rows starting at row r0, lm_head
 // into logits rows lrow.., argmax into next rows lrow...
-q2_status run_head(q2_model* M, int r0, int rows, int lrow, cudaStream_t st, bool pdl) {
+q2_status run_head(q2_model* M, int r0, int rows, int lrow, cudaStream_t st, bool pdl,
+                   bool add_o = true) {
   const q2_meta& m = M->m;
   const int H = m.hidden, V = m.vocab, dt = M->dt;
   char* x = (char*)M->x + (size_t)r0 * H * M->es;
-  char* o = (char*)M->o + (size_t)r0 * H * M->es;
+  char* o = add_o ? (char*)M->o + (size_t)r0 * H * M->es : nullptr;
   char* h = (char*)M->h + (size_t)r0 * H * M->es;
   TIMED(Q2_K_NORM, launch_add_rms_norm(x, o, h, M->final_norm, rows, H, m.eps, dt, st, pdl));
   float* lg = M->logits + (size_t)lrow * V;
@@ -792,6 +793,48 @@ q2_status q2_model_time_kernels(q2_model* M, const int64_t* ids, int B, int step
     mean_ms[c] = cnt[c] ? (float)(sum[c] / ((double)cnt[c] * steps)) : 0.f;
   }
   *kernels_per_step = t->kernels;
+  return Q2_OK;
+}
+
+q2_status q2_model_prefill_hidden(q2_model* M, int seq, const void* x_in, int T, void* x_out,
+                                  void* stream) {
+  clear_error();
+  Q2_CHECK_ARG(M && x_in && x_out, Q2_ERR_INVALID_ARG, "prefill_hidden: NULL argument");
+  Q2_CHECK_ARG(seq >= 0 && seq < M->m.max_batch, Q2_ERR_INVALID_ARG, "prefill_hidden: bad sequence");
+  Q2_CHECK_ARG(T >= 1, Q2_ERR_INVALID_ARG, "prefill_hidden: T must be positive");
+  Q2_CHECK_ARG((long long)M->h_len[seq] + T <= M->m.max_seq, Q2_ERR_CAPACITY,
+               "prefill_hidden: the sequence would pass max_seq");
+  DeviceGuard g(M->device);
+  cudaStream_t st = as_stream(stream);
+  Q2_TRY(check_stream_device(M, st));
+  const size_t row = (size_t)M->m.hidden * M->es;
+  for (int c = 0; c < T; c += M->chunk) {
+    const int Tc = T - c < M->chunk ? T - c : M->chunk;
+    const int pos0 = M->h_len[seq];
+    Q2_CUDA_TRY(cudaMemcpyAsync(M->x, (const char*)x_in + c * row, Tc * row, cudaMemcpyDeviceToDevice, st));
+    Q2_TRY(run_layers(M, Tc, 0, seq, pos0, st, true));
+    Q2_TRY(launch_add_rms_norm(M->x, M->o, nullptr, nullptr, Tc, M->m.hidden, M->m.eps, M->dt, st, true));
+    Q2_CUDA_TRY(cudaMemcpyAsync((char*)x_out + c * row, M->x, Tc * row, cudaMemcpyDeviceToDevice, st));
+    M->h_len[seq] = pos0 + Tc;
+    Q2_LAUNCH(set_len_kernel, dim3(1), dim3(1), 0, st, true, M->d_len, seq, pos0 + Tc);
+  }
+  return Q2_OK;
+}
+
+q2_status q2_model_head(q2_model* M, const void* x, int rows, int64_t* next, float* logits,
+                        void* stream) {
+  clear_error();
+  Q2_CHECK_ARG(M && x && next, Q2_ERR_INVALID_ARG, "head: NULL argument");
+  Q2_CHECK_ARG(rows >= 1 && rows <= M->m.max_batch, Q2_ERR_CAPACITY, "head: rows outside [1, max_batch]");
+  DeviceGuard g(M->device);
+  cudaStream_t st = as_stream(stream);
+  Q2_TRY(check_stream_device(M, st));
+  Q2_CUDA_TRY(cudaMemcpyAsync(M->x, x, (size_t)rows * M->m.hidden * M->es, cudaMemcpyDeviceToDevice, st));
+  Q2_TRY(run_head(M, 0, rows, 0, st, true, false));
+  Q2_CUDA_TRY(cudaMemcpyAsync(next, M->d_next, rows * sizeof(int64_t), cudaMemcpyDeviceToDevice, st));
+  if (logits)
+    Q2_CUDA_TRY(cudaMemcpyAsync(logits, M->logits, (size_t)rows * M->m.vocab * sizeof(float),
+                                cudaMemcpyDeviceToDevice, st));
   return Q2_OK;
 }
 
