@@ -84,6 +84,28 @@ q2_status q2_add(void* c, const void* a, const void* b, size_t n, int dtype, voi
 q2_status q2_argmax(int64_t* max_idx, void* max_val, const void* vals, size_t rows, size_t n,
                     int dtype, void* stream);
 
+/* q2_argmax without any device allocation (the pages have no counterpart:
+ * an addition of this library).  Same arguments and results as q2_argmax,
+ * for callers that must not have a library allocate device memory at the
+ * moment they call it -- a host that hands all device memory to its own pool
+ * and passes only its inputs and outputs, a latency-critical loop that must
+ * not wait on the allocator, or code recording into a CUDA graph under a
+ * capture mode that refuses allocation calls.  The pass-1 partials live in
+ * a fixed 192 KiB array in the library's device memory (every GPU that
+ * loads the library holds one until the process exits); the call makes no
+ * cudaMalloc/cudaFree or other allocating call.
+ * Limits: rows <= 16384 (rows x partials <= 16384 entries); larger inputs
+ * return Q2_ERR_CAPACITY before any launch.
+ * Set-up: the first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current) and caches it; make that
+ * first call before any stream capture.
+ * Sharing: all calls on a device use the same array and it keeps the last
+ * call's partials.  Nothing in it needs to start at zero (pass 1 writes every
+ * partial that pass 2 reads), but calls whose kernels overlap on the GPU
+ * (different streams, no ordering between them) race on it: order them. */
+q2_status q2_argmax_noalloc(int64_t* max_idx, void* max_val, const void* vals, size_t rows,
+                            size_t n, int dtype, void* stream);
+
 /* embedding: out[t, :] = weight[ids[t], :] for t < ntok; weight [vocab, d],
  * out [ntok, d].  An id outside [0, vocab) writes a zero row and sets the
  * device error flag (see q2_check_device_error). */

@@ -18,7 +18,8 @@ from typing import Dict, Iterable, Optional, Sequence, Tuple
 import torch
 
 __all__ = [
-    "Q2Error", "lib", "q2_version", "q2_check_device_error", "q2_add", "q2_argmax", "q2_embedding",
+    "Q2Error", "lib", "q2_version", "q2_check_device_error", "q2_add", "q2_argmax",
+    "q2_argmax_noalloc", "q2_embedding",
     "q2_linear", "q2_rms_norm", "q2_add_rms_norm", "q2_rope", "q2_self_attention", "q2_swiglu",
     "q2_rearrange", "Model", "W_KIND", "STATUS", "KCLASS",
 ]
@@ -56,6 +57,7 @@ _SIGS = {
     "q2_check_device_error": [_VP],
     "q2_add": [_VP, _VP, _VP, _SZ, _I, _VP],
     "q2_argmax": [_VP, _VP, _VP, _SZ, _SZ, _I, _VP],
+    "q2_argmax_noalloc": [_VP, _VP, _VP, _SZ, _SZ, _I, _VP],
     "q2_embedding": [_VP, _VP, _VP, _SZ, _SZ, _SZ, _I, _VP],
     "q2_linear": [_VP, _VP, _VP, _VP, _SZ, _SZ, _SZ, _I, _VP],
     "q2_rms_norm": [_VP, _VP, _VP, _SZ, _SZ, _F, _I, _VP],
@@ -161,6 +163,16 @@ def q2_argmax(max_idx, max_val, vals):
     rows = 1 if vals.dim() == 1 else vals.shape[0]
     n = vals.shape[-1]
     _call("q2_argmax", _p(max_idx), _p(max_val), _p(vals), rows, n, _dtype(vals), _stream())
+    return max_idx, max_val
+
+
+def q2_argmax_noalloc(max_idx, max_val, vals):
+    """q2_argmax with no device allocation (fixed library-owned partials array;
+    rows <= 16384).  Same arguments as q2_argmax."""
+    _dense(vals, max_idx, max_val)
+    rows = 1 if vals.dim() == 1 else vals.shape[0]
+    n = vals.shape[-1]
+    _call("q2_argmax_noalloc", _p(max_idx), _p(max_val), _p(vals), rows, n, _dtype(vals), _stream())
     return max_idx, max_val
 
 
