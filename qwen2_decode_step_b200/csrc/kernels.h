@@ -17,9 +17,9 @@ size_t dtype_size(int dtype);
 q2_status launch_add(void* c, const void* a, const void* b, size_t n, int dtype, cudaStream_t st);
 q2_status launch_swiglu(void* out, const void* gate, const void* up, size_t n, int dtype,
                         cudaStream_t st);
-// out[t, :] = gate_up[t, 0:I] -> silu, times gate_up[t, I:2I]; rows of stride 2I.
-q2_status launch_swiglu_rows(void* out, const void* gate_up, int T, int I, int dtype,
-                             cudaStream_t st, bool pdl);
+// out[t, i] = silu(gate_up[t, 2i]) * gate_up[t, 2i+1]; rows of stride 2I.
+q2_status launch_swiglu_interleaved(void* out, const void* gate_up, int T, int I, int dtype,
+                                    cudaStream_t st, bool pdl);
 q2_status launch_embedding(void* out, const int64_t* ids, const void* table, size_t ntok,
                            size_t vocab, size_t d, int dtype, int* err_flag, cudaStream_t st,
                            bool pdl);

@@ -16,18 +16,26 @@
 #include <vector>
 
 #include "common.cuh"
+#include "decode.h"
 #include "kernels.h"
+#include "tma.h"
 
 using namespace q2;
 
+// Packed weight layouts (the library repacks on load):
+//  wqkv [nh*hd + 2*nkv*hd, H]: head slots (q heads, then k heads, then v
+//       heads); inside a slot, row 2j holds original row j and row 2j+1
+//       original row j + hd/2, so the two members of a RoPE pair are adjacent
+//       rows (one fused-epilogue stage sees both).  bqkv the same way.
+//  wgu  [2I, H]: row 2i = gate row i, row 2i+1 = up row i.
 struct LayerW {
   void* in_norm;
-  void* wqkv;  // [nh*hd + 2*nkv*hd, H]: q rows, then k rows, then v rows
-  void* bqkv;  // [nh*hd + 2*nkv*hd]
+  void* wqkv;
+  void* bqkv;
   void* wo;    // [H, nh*hd]
   void* post_norm;
-  void* wgu;  // [2I, H]: gate rows, then up rows
-  void* wd;   // [H, I]
+  void* wgu;
+  void* wd;    // [H, I]
 };
 
 // Event pairs around kernel-class instances, for q2_model_time_kernels.
@@ -58,8 +66,8 @@ struct q2_model {
   int* d_len = nullptr;
   std::vector<int> h_len;
 
-  void *x = nullptr, *h = nullptr, *qkv = nullptr, *att = nullptr, *o = nullptr, *gu = nullptr,
-       *s = nullptr;
+  void *x = nullptr, *h = nullptr, *qkv = nullptr, *qb = nullptr, *att = nullptr, *o = nullptr,
+       *gu = nullptr, *s = nullptr;
   float* logits = nullptr;
   int64_t* d_ids = nullptr;
   int64_t* d_next = nullptr;
@@ -68,7 +76,12 @@ struct q2_model {
   float* am_val = nullptr;
   int64_t* am_idx = nullptr;
   int* d_err = nullptr;
+  unsigned* d_counters = nullptr;  // [max_batch * nkv] attention + [1] lm_head (zero between launches)
+  float* lm_val = nullptr;         // lm_head per-CTA argmax partials [num_sms][kDecodeMaxBatch]
+  int64_t* lm_idx = nullptr;
   void* abuf = nullptr;
+  bool fused = false;              // bf16 and the fused decode kernels support the shapes
+  CUtensorMap kmap{}, vmap{};      // the K and V caches as 2-D [rows, hd] tensors
 
   cudaStream_t cap = nullptr;
   bool use_graphs = true;
@@ -127,9 +140,9 @@ void tend(q2_model* M, cudaStream_t st) {
 // next position of sequence t.  Prefill: token t is position pos0 + t of
 // sequence `seq`.
 template <typename T>
-__global__ void rope_kv_kernel(T* qkv, int qkvd, int T_, int nh, int nkv, int hd, const float2* rope,
-                               T* kc, T* vc, long long kv_seq_stride, int max_seq, const int* lens,
-                               int decode, int seq, int pos0) {
+__global__ void rope_kv_kernel(const T* qkv, int qkvd, T* qb, int qd, int T_, int nh, int nkv, int hd,
+                               const float2* rope, T* kc, T* vc, long long kv_seq_stride, int max_seq,
+                               const int* lens, int decode, int seq, int pos0) {
   pdl_launch_dependents();
   pdl_wait();
   const int half = hd >> 1;
@@ -142,24 +155,20 @@ __global__ void rope_kv_kernel(T* qkv, int qkvd, int T_, int nh, int nkv, int hd
     const int t = (int)(i / ((long long)half * heads));
     const int sq = decode ? t : seq;
     const int pos = decode ? lens[t] : pos0 + t;
-    T* row = qkv + (size_t)t * qkvd + (size_t)hh * hd;
-    const float a = to_f(row[j]), b = to_f(row[j + half]);
+    const T* row = qkv + (size_t)t * qkvd + (size_t)hh * hd;  // packed: pair j at 2j, 2j+1
+    const float a = to_f(row[2 * j]), b = to_f(row[2 * j + 1]);
     if (hh < nh + nkv) {
       const float2 cs = rope[(size_t)pos * half + j];
       const T ra = from_f<T>(a * cs.x - b * cs.y);
       const T rb = from_f<T>(b * cs.x + a * cs.y);
-      if (hh < nh) {
-        row[j] = ra;
-        row[j + half] = rb;
-      } else {
-        T* dst = kc + (size_t)sq * kv_seq_stride + ((size_t)(hh - nh) * max_seq + pos) * hd;
-        dst[j] = ra;
-        dst[j + half] = rb;
-      }
+      T* dst = hh < nh ? qb + (size_t)t * qd + (size_t)hh * hd
+                       : kc + (size_t)sq * kv_seq_stride + ((size_t)(hh - nh) * max_seq + pos) * hd;
+      dst[j] = ra;
+      dst[j + half] = rb;
     } else {
       T* dst = vc + (size_t)sq * kv_seq_stride + ((size_t)(hh - nh - nkv) * max_seq + pos) * hd;
-      dst[j] = row[j];
-      dst[j + half] = row[j + half];
+      dst[j] = row[2 * j];
+      dst[j + half] = row[2 * j + 1];
     }
   }
 }
@@ -185,15 +194,15 @@ q2_status launch_rope_kv(q2_model* M, int l, int T, const int* lens, int decode,
   if (blocks < 1) blocks = 1;
   size_t loff = (size_t)l * M->kv_layer_stride;
   if (M->dt == Q2_F32)
-    Q2_LAUNCH(rope_kv_kernel<float>, dim3(blocks), dim3(256), 0, st, pdl, (float*)M->qkv, M->qkvd,
-              T, m.n_heads, m.n_kv_heads, m.head_dim, (const float2*)M->rope,
-              (float*)M->kc + loff, (float*)M->vc + loff, M->kv_seq_stride, m.max_seq, lens, decode,
-              seq, pos0);
+    Q2_LAUNCH(rope_kv_kernel<float>, dim3(blocks), dim3(256), 0, st, pdl, (const float*)M->qkv,
+              M->qkvd, (float*)M->qb, M->qd, T, m.n_heads, m.n_kv_heads, m.head_dim,
+              (const float2*)M->rope, (float*)M->kc + loff, (float*)M->vc + loff, M->kv_seq_stride,
+              m.max_seq, lens, decode, seq, pos0);
   else
     Q2_LAUNCH(rope_kv_kernel<__nv_bfloat16>, dim3(blocks), dim3(256), 0, st, pdl,
-              (__nv_bfloat16*)M->qkv, M->qkvd, T, m.n_heads, m.n_kv_heads, m.head_dim,
-              (const float2*)M->rope, (__nv_bfloat16*)M->kc + loff, (__nv_bfloat16*)M->vc + loff,
-              M->kv_seq_stride, m.max_seq, lens, decode, seq, pos0);
+              (const __nv_bfloat16*)M->qkv, M->qkvd, (__nv_bfloat16*)M->qb, M->qd, T, m.n_heads,
+              m.n_kv_heads, m.head_dim, (const float2*)M->rope, (__nv_bfloat16*)M->kc + loff,
+              (__nv_bfloat16*)M->vc + loff, M->kv_seq_stride, m.max_seq, lens, decode, seq, pos0);
   return Q2_OK;
 }
 
@@ -215,8 +224,8 @@ q2_status run_layers(q2_model* M, int T, int decode, int seq, int pos0, cudaStre
     TIMED(Q2_K_ROPE_KV, launch_rope_kv(M, l, T, M->d_len, decode, seq, pos0, st, pdl));
 
     AttnRows a = {};
-    a.q = M->qkv;
-    a.q_row_stride = M->qkvd;
+    a.q = M->qb;
+    a.q_row_stride = M->qd;
     size_t loff = (size_t)l * M->kv_layer_stride * M->es;
     a.k = (const char*)M->kc + loff;
     a.v = (const char*)M->vc + loff;
@@ -251,7 +260,7 @@ q2_status run_layers(q2_model* M, int T, int decode, int seq, int pos0, cudaStre
     TIMED(Q2_K_O, launch_linear(M->o, M->att, w.wo, nullptr, T, H, M->qd, dt, dt, st, pdl));
     TIMED(Q2_K_NORM, launch_add_rms_norm(M->x, M->o, M->h, w.post_norm, T, H, m.eps, dt, st, pdl));
     TIMED(Q2_K_GATE_UP, launch_linear(M->gu, M->h, w.wgu, nullptr, T, 2 * I, H, dt, dt, st, pdl));
-    TIMED(Q2_K_SWIGLU, launch_swiglu_rows(M->s, M->gu, T, I, dt, st, pdl));
+    TIMED(Q2_K_SWIGLU, launch_swiglu_interleaved(M->s, M->gu, T, I, dt, st, pdl));
     TIMED(Q2_K_DOWN, launch_linear(M->o, M->s, w.wd, nullptr, T, H, I, dt, dt, st, pdl));
     if (l + 1 < m.n_layers)
       TIMED(Q2_K_NORM,
@@ -278,7 +287,130 @@ q2_status run_head(q2_model* M, int r0, int rows, int lrow, cudaStream_t st, boo
   return Q2_OK;
 }
 
+// ---- the fused bf16 decode path (batch <= kDecodeMaxBatch): five kernels
+// per layer, norms/RoPE/KV append/SwiGLU/residual adds in the linears'
+// prologues and epilogues, split attention with its combine folded in.
+bool use_fused(const q2_model* M, int B) { return M->fused && B >= 1 && B <= kDecodeMaxBatch; }
+
+q2_status fused_layers(q2_model* M, int B, cudaStream_t st) {
+  const q2_meta& m = M->m;
+  const int H = m.hidden, I = m.intermediate;
+  const int nsplit = decode_splits(M, B);
+  for (int l = 0; l < m.n_layers; ++l) {
+    const LayerW& w = M->layers[l];
+    const size_t loff = (size_t)l * M->kv_layer_stride * M->es;
+    DGemv q = {};
+    q.w = w.wqkv;
+    q.N = M->qkvd;
+    q.K = H;
+    q.M = B;
+    q.x = M->x;
+    q.norm_w = w.in_norm;
+    q.eps = m.eps;
+    q.bias = w.bqkv;
+    q.out = M->qb;
+    q.out_stride = M->qd;
+    q.kc = (char*)M->kc + loff;
+    q.vc = (char*)M->vc + loff;
+    q.kv_seq_stride = M->kv_seq_stride;
+    q.max_seq = m.max_seq;
+    q.rope = M->rope;
+    q.lens = M->d_len;
+    q.nh = m.n_heads;
+    q.nkv = m.n_kv_heads;
+    q.hd = m.head_dim;
+    q.err = M->d_err;
+    TIMED(Q2_K_QKV, launch_dgemv(EPI_QKV, q, st));
+
+    DAttn a = {};
+    a.q = M->qb;
+    a.q_stride = M->qd;
+    a.out = M->att;
+    a.part_o = (float*)M->attn_scratch;
+    a.part_ml = a.part_o + (size_t)B * m.n_heads * nsplit * m.head_dim;
+    a.counters = M->d_counters;
+    a.lens = M->d_len;
+    a.B = B;
+    a.nh = m.n_heads;
+    a.nkv = m.n_kv_heads;
+    a.hd = m.head_dim;
+    a.nsplit = nsplit;
+    a.max_seq = m.max_seq;
+    a.Bmax = m.max_batch;
+    a.layer = l;
+    a.scale = 1.0f / sqrtf((float)m.head_dim);
+    a.err = M->d_err;
+    TIMED(Q2_K_ATTN, launch_dattn(a, M->kmap, M->vmap, st));
+
+    DGemv o = {};
+    o.w = w.wo;
+    o.N = H;
+    o.K = M->qd;
+    o.M = B;
+    o.x = M->att;
+    o.out = M->x;
+    o.out_stride = H;
+    o.err = M->d_err;
+    TIMED(Q2_K_O, launch_dgemv(EPI_RESID, o, st));
+
+    DGemv gu = {};
+    gu.w = w.wgu;
+    gu.N = 2 * I;
+    gu.K = H;
+    gu.M = B;
+    gu.x = M->x;
+    gu.norm_w = w.post_norm;
+    gu.eps = m.eps;
+    gu.out = M->s;
+    gu.out_stride = I;
+    gu.err = M->d_err;
+    TIMED(Q2_K_GATE_UP, launch_dgemv(EPI_SWIGLU, gu, st));
+
+    DGemv dn = {};
+    dn.w = w.wd;
+    dn.N = H;
+    dn.K = I;
+    dn.M = B;
+    dn.x = M->s;
+    dn.out = M->x;
+    dn.out_stride = H;
+    dn.err = M->d_err;
+    TIMED(Q2_K_DOWN, launch_dgemv(EPI_RESID, dn, st));
+  }
+  return Q2_OK;
+}
+
+q2_status fused_head(q2_model* M, int B, cudaStream_t st) {
+  const q2_meta& m = M->m;
+  DGemv h = {};
+  h.w = M->lm_head;
+  h.N = m.vocab;
+  h.K = m.hidden;
+  h.M = B;
+  h.x = M->x;
+  h.norm_w = M->final_norm;
+  h.eps = m.eps;
+  h.logits = M->logits;
+  h.am_val = M->lm_val;
+  h.am_idx = M->lm_idx;
+  h.counter = M->d_counters + (size_t)m.max_batch * m.n_kv_heads;
+  h.next = M->d_next;
+  h.lens_inc = M->d_len;
+  h.err = M->d_err;
+  TIMED(Q2_K_LM_HEAD, launch_dgemv(EPI_LOGITS, h, st));
+  return Q2_OK;
+}
+
+q2_status decode_body_fused(q2_model* M, int B, cudaStream_t st) {
+  const q2_meta& m = M->m;
+  TIMED(Q2_K_EMBED,
+        launch_embedding(M->x, M->d_ids, M->embed, B, m.vocab, m.hidden, M->dt, M->d_err, st, true));
+  Q2_TRY(fused_layers(M, B, st));
+  return fused_head(M, B, st);
+}
+
 q2_status decode_body(q2_model* M, int B, cudaStream_t st) {
+  if (use_fused(M, B)) return decode_body_fused(M, B, st);
   const bool pdl = true;
   const q2_meta& m = M->m;
   TIMED(Q2_K_EMBED,
@@ -439,6 +571,12 @@ q2_status q2_model_create(const q2_meta* meta, int device, q2_model** out) {
     size_t b = attn_scratch_bytes(r, m.n_heads, m.head_dim, attn_splits(r, m.n_kv_heads, m.max_seq));
     if (b > scratch) scratch = b;
   }
+  // The fused decode attention always writes split partials (even with one split).
+  for (int r = 1; r <= m.max_batch && r <= kDecodeMaxBatch; ++r) {
+    const size_t n = (size_t)r * m.n_heads * attn_splits(r, m.n_kv_heads, m.max_seq);
+    const size_t b = n * m.head_dim * sizeof(float) + 2 * n * sizeof(float) + 256;
+    if (b > scratch) scratch = b;
+  }
   size_t am = 0;
   for (int r = 1; r <= m.max_batch; ++r) {
     size_t b = (size_t)r * argmax_parts(r, V);
@@ -448,6 +586,7 @@ q2_status q2_model_create(const q2_meta* meta, int device, q2_model** out) {
   al.push_back({&M->x, T * H * es});
   al.push_back({&M->h, T * H * es});
   al.push_back({&M->qkv, T * M->qkvd * es});
+  al.push_back({&M->qb, T * M->qd * es});
   al.push_back({&M->att, T * M->qd * es});
   al.push_back({&M->o, T * H * es});
   al.push_back({&M->gu, T * 2 * I * es});
@@ -461,6 +600,9 @@ q2_status q2_model_create(const q2_meta* meta, int device, q2_model** out) {
   al.push_back({(void**)&M->am_idx, am * sizeof(int64_t)});
   al.push_back({(void**)&M->d_len, (size_t)m.max_batch * sizeof(int)});
   al.push_back({(void**)&M->d_err, sizeof(int)});
+  al.push_back({(void**)&M->d_counters, ((size_t)m.max_batch * m.n_kv_heads + 16) * sizeof(unsigned)});
+  al.push_back({(void**)&M->lm_val, (size_t)num_sms() * kDecodeMaxBatch * sizeof(float)});
+  al.push_back({(void**)&M->lm_idx, (size_t)num_sms() * kDecodeMaxBatch * sizeof(int64_t)});
   size_t abytes = 0;
   for (auto& p : al) abytes += align_up(p.second ? p.second : 1, 256);
   if (cudaMalloc(&M->abuf, abytes) != cudaSuccess) {
@@ -494,6 +636,20 @@ q2_status q2_model_create(const q2_meta* meta, int device, q2_model** out) {
       set_error("model_create: cannot upload the RoPE table");
       return fail(Q2_ERR_CUDA);
     }
+  }
+  // ---- the fused bf16 decode path: K/V caches as 2-D [rows, hd] tensors for TMA
+  if (m.dtype == Q2_BF16 && dattn_supported(m.n_heads, m.n_kv_heads, m.head_dim) &&
+      dgemv_supported(EPI_QKV, M->qkvd, m.hidden) && dgemv_supported(EPI_RESID, m.hidden, M->qd) &&
+      dgemv_supported(EPI_SWIGLU, 2 * m.intermediate, m.hidden) &&
+      dgemv_supported(EPI_RESID, m.hidden, m.intermediate) &&
+      dgemv_supported(EPI_LOGITS, m.vocab, m.hidden)) {
+    const uint64_t rows = (uint64_t)m.n_layers * m.max_batch * m.n_kv_heads * m.max_seq;
+    const uint64_t pitch = (uint64_t)m.head_dim * 2;
+    q2_status ks = make_tmap_2d_bf16(&M->kmap, M->kc, rows, m.head_dim, pitch, 64, 64, 128);
+    q2_status vs = ks == Q2_OK ? make_tmap_2d_bf16(&M->vmap, M->vc, rows, m.head_dim, pitch, 64, 64, 128)
+                               : ks;
+    M->fused = (vs == Q2_OK) && rows < (1ull << 31);
+    clear_error();
   }
   if (cudaStreamCreateWithFlags(&M->cap, cudaStreamNonBlocking) != cudaSuccess) {
     set_error("model_create: cannot create a stream");
@@ -562,8 +718,40 @@ q2_status q2_model_load_weight(q2_model* M, int kind, int layer, const void* src
   DeviceGuard g(M->device);
   cudaStream_t st = as_stream(stream);
   Q2_TRY(check_stream_device(M, st));
-  Q2_CUDA_TRY(cudaMemcpyAsync(dst, src, nbytes, cudaMemcpyDeviceToDevice, st));
-  return Q2_OK;
+  const char* sp = static_cast<const char*>(src);
+  const size_t hd = m.head_dim, half = hd / 2;
+  switch (kind) {
+    case Q2_W_Q:
+    case Q2_W_K:
+    case Q2_W_V:
+    case Q2_W_Q_BIAS:
+    case Q2_W_K_BIAS:
+    case Q2_W_V_BIAS: {
+      // Head slot by head slot: original rows j < hd/2 go to packed rows 2j,
+      // rows j + hd/2 to packed rows 2j + 1 (a row of a bias is one element).
+      const bool bias = kind == Q2_W_Q_BIAS || kind == Q2_W_K_BIAS || kind == Q2_W_V_BIAS;
+      const size_t row = bias ? es : H * es;
+      const int heads = (kind == Q2_W_Q || kind == Q2_W_Q_BIAS) ? m.n_heads : m.n_kv_heads;
+      for (int hh = 0; hh < heads; ++hh) {
+        char* d = dst + (size_t)hh * hd * row;
+        const char* s0 = sp + (size_t)hh * hd * row;
+        Q2_CUDA_TRY(cudaMemcpy2DAsync(d, 2 * row, s0, row, row, half, cudaMemcpyDeviceToDevice, st));
+        Q2_CUDA_TRY(cudaMemcpy2DAsync(d + row, 2 * row, s0 + half * row, row, row, half,
+                                      cudaMemcpyDeviceToDevice, st));
+      }
+      return Q2_OK;
+    }
+    case Q2_W_GATE:
+    case Q2_W_UP: {
+      // Interleaved rows: gate row i -> packed row 2i, up row i -> 2i + 1.
+      char* d = (char*)L->wgu + (kind == Q2_W_UP ? H * es : 0);
+      Q2_CUDA_TRY(cudaMemcpy2DAsync(d, 2 * H * es, sp, H * es, H * es, I, cudaMemcpyDeviceToDevice, st));
+      return Q2_OK;
+    }
+    default:
+      Q2_CUDA_TRY(cudaMemcpyAsync(dst, src, nbytes, cudaMemcpyDeviceToDevice, st));
+      return Q2_OK;
+  }
 }
 
 q2_status q2_model_decode_step(q2_model* M, const int64_t* ids, int B, int64_t* next, float* logits,
@@ -611,8 +799,12 @@ q2_status q2_model_forward_hidden(q2_model* M, const void* x_in, int B, void* x_
   Q2_TRY(check_stream_device(M, st));
   const size_t bytes = (size_t)B * M->m.hidden * M->es;
   Q2_CUDA_TRY(cudaMemcpyAsync(M->x, x_in, bytes, cudaMemcpyDeviceToDevice, st));
-  Q2_TRY(run_layers(M, B, 1, 0, 0, st, false));
-  Q2_TRY(launch_add_rms_norm(M->x, M->o, nullptr, nullptr, B, M->m.hidden, M->m.eps, M->dt, st, false));
+  if (use_fused(M, B)) {
+    Q2_TRY(fused_layers(M, B, st));  // the residual stream ends in x
+  } else {
+    Q2_TRY(run_layers(M, B, 1, 0, 0, st, false));
+    Q2_TRY(launch_add_rms_norm(M->x, M->o, nullptr, nullptr, B, M->m.hidden, M->m.eps, M->dt, st, false));
+  }
   Q2_CUDA_TRY(cudaMemcpyAsync(x_out, M->x, bytes, cudaMemcpyDeviceToDevice, st));
   Q2_LAUNCH(inc_lens_kernel, dim3(1), dim3(64 * ((B + 63) / 64)), 0, st, false, M->d_len, B);
   for (int b = 0; b < B; ++b) M->h_len[b] += 1;

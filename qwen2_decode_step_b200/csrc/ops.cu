@@ -91,28 +91,28 @@ q2_status launch_swiglu(void* out, const void* gate, const void* up, size_t n, i
   return Q2_OK;
 }
 
-// Rows of [gate | up] (stride 2I) -> out [T, I].
+// Rows of interleaved gate/up values (row stride 2I: element 2i is gate i,
+// element 2i+1 is up i) -> out [T, I].
 template <typename T>
-__global__ void swiglu_rows_kernel(T* out, const T* gu, int I) {
+__global__ void swiglu_interleaved_kernel(T* out, const T* gu, int I) {
   pdl_launch_dependents();
   pdl_wait();
   int t = blockIdx.y;
   const T* g = gu + (size_t)t * 2 * I;
-  const T* u = g + I;
   T* o = out + (size_t)t * I;
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < I; i += gridDim.x * blockDim.x)
-    o[i] = from_f<T>(silu_mul(to_f(g[i]), to_f(u[i])));
+    o[i] = from_f<T>(silu_mul(to_f(g[2 * i]), to_f(g[2 * i + 1])));
 }
 
-q2_status launch_swiglu_rows(void* out, const void* gu, int T, int I, int dtype, cudaStream_t st,
-                             bool pdl) {
+q2_status launch_swiglu_interleaved(void* out, const void* gu, int T, int I, int dtype,
+                                    cudaStream_t st, bool pdl) {
   if (T == 0) return Q2_OK;
   dim3 grid(ceil_div(I, 256) > 64 ? 64 : ceil_div(I, 256), T);
   if (dtype == Q2_F32)
-    Q2_LAUNCH(swiglu_rows_kernel<float>, grid, dim3(256), 0, st, pdl, (float*)out,
+    Q2_LAUNCH(swiglu_interleaved_kernel<float>, grid, dim3(256), 0, st, pdl, (float*)out,
               (const float*)gu, I);
   else
-    Q2_LAUNCH(swiglu_rows_kernel<__nv_bfloat16>, grid, dim3(256), 0, st, pdl,
+    Q2_LAUNCH(swiglu_interleaved_kernel<__nv_bfloat16>, grid, dim3(256), 0, st, pdl,
               (__nv_bfloat16*)out, (const __nv_bfloat16*)gu, I);
   return Q2_OK;
 }
