@@ -294,6 +294,22 @@ q2_status q2_model_check_error(q2_model* model, void* stream);
  * launches, for debugging and per-kernel timing). */
 q2_status q2_model_set_graphs(q2_model* model, int enable);
 
+/* Decode-step implementation for bf16 models at batch <= 4:
+ * Q2_PATH_AUTO (default: the fused per-layer kernels where the shapes allow),
+ * Q2_PATH_PERSISTENT (one cooperative launch per step: every CTA streams its
+ * share of all weights through one TMA ring while the phases of the step run
+ * between grid-wide counters), Q2_PATH_KERNELS (five fused kernels per layer
+ * chained by programmatic dependent launch), Q2_PATH_GENERIC (one kernel per
+ * operator).  Larger batches and fp32 models always take the generic path.
+ * Q2_ERR_STATE if the requested path is not available for this model. */
+typedef enum q2_path {
+  Q2_PATH_AUTO = 0,
+  Q2_PATH_PERSISTENT = 1,
+  Q2_PATH_KERNELS = 2,
+  Q2_PATH_GENERIC = 3
+} q2_path;
+q2_status q2_model_set_decode_path(q2_model* model, int path);
+
 /* Kernel classes of a decode step, for q2_model_time_kernels. */
 typedef enum q2_kclass {
   Q2_K_EMBED = 0,   /* embedding gather */
@@ -308,7 +324,8 @@ typedef enum q2_kclass {
   Q2_K_LM_HEAD = 9, /* final norm + lm_head linear */
   Q2_K_ARGMAX = 10, /* argmax over the vocabulary */
   Q2_K_OTHER = 11,  /* length bookkeeping */
-  Q2_K_COUNT = 12
+  Q2_K_STEP = 12,   /* the whole step as one persistent kernel */
+  Q2_K_COUNT = 13
 } q2_kclass;
 
 /* Per-kernel device timing of decode steps.  Captures (once per batch size)

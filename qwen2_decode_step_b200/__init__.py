@@ -82,10 +82,12 @@ _SIGS = {
     "q2_model_time_kernels": [_VP, _VP, _I, _I, _VP, _VP, ctypes.POINTER(_I), _VP],
     "q2_model_prefill_hidden": [_VP, _I, _VP, _I, _VP, _VP],
     "q2_model_head": [_VP, _VP, _I, _VP, _VP, _VP],
+    "q2_model_set_decode_path": [_VP, _I],
 }
 
 KCLASS = ["embed", "norm", "qkv", "rope_kv", "attn", "o", "gate_up", "swiglu", "down", "lm_head",
-          "argmax", "other"]
+          "argmax", "other", "step"]
+PATH = {"auto": 0, "persistent": 1, "kernels": 2, "generic": 3}
 
 _lib = None
 
@@ -374,6 +376,10 @@ class Model:
 
     def set_graphs(self, enable: bool):
         _call("q2_model_set_graphs", self._h, 1 if enable else 0)
+
+    def set_decode_path(self, path: str):
+        """'auto' | 'persistent' | 'kernels' | 'generic' (q2_model_set_decode_path)."""
+        _call("q2_model_set_decode_path", self._h, PATH[path])
 
     def time_kernels(self, ids: torch.Tensor, steps: int):
         """Per kernel class: (mean ms per instance, instances per step), plus the

@@ -18,6 +18,7 @@
 #include "common.cuh"
 #include "decode.h"
 #include "kernels.h"
+#include "pdecode.h"
 #include "tma.h"
 
 using namespace q2;
@@ -81,6 +82,11 @@ struct q2_model {
   int64_t* lm_idx = nullptr;
   void* abuf = nullptr;
   bool fused = false;              // bf16 and the fused decode kernels support the shapes
+  bool persistent = false;         // ... and the persistent decode kernel does too
+  int path = Q2_PATH_AUTO;
+  PLayer* d_layers = nullptr;      // device copy of the per-layer weight pointers
+  unsigned* d_sync = nullptr;      // persistent step phase counters
+  unsigned long long* d_trace = nullptr;  // persistent step phase timestamps [5L + 1][4]
   CUtensorMap kmap{}, vmap{};      // the K and V caches as 2-D [rows, hd] tensors
 
   cudaStream_t cap = nullptr;
@@ -290,7 +296,65 @@ q2_status run_head(q2_model* M, int r0, int rows, int lrow, cudaStream_t st, boo
 // ---- the fused bf16 decode path (batch <= kDecodeMaxBatch): five kernels
 // per layer, norms/RoPE/KV append/SwiGLU/residual adds in the linears'
 // prologues and epilogues, split attention with its combine folded in.
-bool use_fused(const q2_model* M, int B) { return M->fused && B >= 1 && B <= kDecodeMaxBatch; }
+bool use_persistent(const q2_model* M, int B) {
+  return M->persistent && B >= 1 && B <= kPMaxBatch && M->path == Q2_PATH_PERSISTENT;
+}
+bool use_fused(const q2_model* M, int B) {
+  return M->fused && B >= 1 && B <= kDecodeMaxBatch && M->path != Q2_PATH_GENERIC;
+}
+
+// The whole step (or the layers alone) as one persistent cooperative launch.
+q2_status persistent_step(q2_model* M, int B, bool head, bool embed_in, cudaStream_t st,
+                          bool trace = false) {
+  const q2_meta& m = M->m;
+  PDecode p = {};
+  p.layers = M->d_layers;
+  p.L = m.n_layers;
+  p.H = m.hidden;
+  p.I = m.intermediate;
+  p.V = m.vocab;
+  p.nh = m.n_heads;
+  p.nkv = m.n_kv_heads;
+  p.hd = m.head_dim;
+  p.qkvd = M->qkvd;
+  p.qd = M->qd;
+  p.max_seq = m.max_seq;
+  p.Bmax = m.max_batch;
+  p.B = B;
+  p.nsplit = decode_splits(M, B);
+  p.eps = m.eps;
+  p.scale = 1.0f / sqrtf((float)m.head_dim);
+  p.embed_in = embed_in ? 1 : 0;
+  p.run_head = head ? 1 : 0;
+  p.embed = M->embed;
+  p.lm_head = M->lm_head;
+  p.final_norm = M->final_norm;
+  p.ids = M->d_ids;
+  p.x = M->x;
+  p.qb = M->qb;
+  p.s = M->s;
+  p.kc = M->kc;
+  p.vc = M->vc;
+  p.kv_layer_stride = M->kv_layer_stride;
+  p.kv_seq_stride = M->kv_seq_stride;
+  p.rope = M->rope;
+  p.lens = M->d_len;
+  p.part_o = (float*)M->attn_scratch;
+  p.part_ml = p.part_o + (size_t)B * m.n_heads * p.nsplit * m.head_dim;
+  p.logits = M->logits;
+  p.am_val = M->lm_val;
+  p.am_idx = M->lm_idx;
+  p.next = M->d_next;
+  p.att = M->att;
+  p.sync = M->d_sync;
+  p.trace = trace ? M->d_trace : nullptr;
+  p.err = M->d_err;
+  Q2_CUDA_TRY(cudaMemsetAsync(M->d_sync, 0, pdecode_sync_words(m.n_layers) * sizeof(unsigned), st));
+  if (trace)
+    Q2_CUDA_TRY(cudaMemsetAsync(M->d_trace, 0, (5 * (size_t)m.n_layers + 1) * 4 * sizeof(unsigned long long), st));
+  TIMED(Q2_K_STEP, launch_pdecode(p, M->kmap, M->vmap, st));
+  return Q2_OK;
+}
 
 q2_status fused_layers(q2_model* M, int B, cudaStream_t st) {
   const q2_meta& m = M->m;
@@ -410,6 +474,7 @@ q2_status decode_body_fused(q2_model* M, int B, cudaStream_t st) {
 }
 
 q2_status decode_body(q2_model* M, int B, cudaStream_t st) {
+  if (use_persistent(M, B)) return persistent_step(M, B, true, true, st);
   if (use_fused(M, B)) return decode_body_fused(M, B, st);
   const bool pdl = true;
   const q2_meta& m = M->m;
@@ -603,6 +668,9 @@ q2_status q2_model_create(const q2_meta* meta, int device, q2_model** out) {
   al.push_back({(void**)&M->d_counters, ((size_t)m.max_batch * m.n_kv_heads + 16) * sizeof(unsigned)});
   al.push_back({(void**)&M->lm_val, (size_t)num_sms() * kDecodeMaxBatch * sizeof(float)});
   al.push_back({(void**)&M->lm_idx, (size_t)num_sms() * kDecodeMaxBatch * sizeof(int64_t)});
+  al.push_back({(void**)&M->d_sync, pdecode_sync_words(m.n_layers) * sizeof(unsigned)});
+  al.push_back({(void**)&M->d_layers, (size_t)m.n_layers * sizeof(PLayer)});
+  al.push_back({(void**)&M->d_trace, (5 * (size_t)m.n_layers + 1) * 4 * sizeof(unsigned long long)});
   size_t abytes = 0;
   for (auto& p : al) abytes += align_up(p.second ? p.second : 1, 256);
   if (cudaMalloc(&M->abuf, abytes) != cudaSuccess) {
@@ -649,7 +717,21 @@ q2_status q2_model_create(const q2_meta* meta, int device, q2_model** out) {
     q2_status vs = ks == Q2_OK ? make_tmap_2d_bf16(&M->vmap, M->vc, rows, m.head_dim, pitch, 64, 64, 128)
                                : ks;
     M->fused = (vs == Q2_OK) && rows < (1ull << 31);
+    M->persistent = M->fused && pdecode_supported(m.hidden, m.intermediate, m.vocab, m.n_heads,
+                                                  m.n_kv_heads, m.head_dim, M->qkvd, M->qd);
     clear_error();
+  }
+  {
+    std::vector<PLayer> pl(m.n_layers);
+    for (int l = 0; l < m.n_layers; ++l) {
+      const LayerW& w = M->layers[l];
+      pl[l] = PLayer{w.in_norm, w.wqkv, w.bqkv, w.wo, w.post_norm, w.wgu, w.wd};
+    }
+    if (cudaMemcpy(M->d_layers, pl.data(), pl.size() * sizeof(PLayer), cudaMemcpyHostToDevice) !=
+        cudaSuccess) {
+      set_error("model_create: cannot upload the layer table");
+      return fail(Q2_ERR_CUDA);
+    }
   }
   if (cudaStreamCreateWithFlags(&M->cap, cudaStreamNonBlocking) != cudaSuccess) {
     set_error("model_create: cannot create a stream");
@@ -799,6 +881,12 @@ q2_status q2_model_forward_hidden(q2_model* M, const void* x_in, int B, void* x_
   Q2_TRY(check_stream_device(M, st));
   const size_t bytes = (size_t)B * M->m.hidden * M->es;
   Q2_CUDA_TRY(cudaMemcpyAsync(M->x, x_in, bytes, cudaMemcpyDeviceToDevice, st));
+  if (use_persistent(M, B)) {
+    Q2_TRY(persistent_step(M, B, false, false, st));  // advances the lengths itself
+    Q2_CUDA_TRY(cudaMemcpyAsync(x_out, M->x, bytes, cudaMemcpyDeviceToDevice, st));
+    for (int b = 0; b < B; ++b) M->h_len[b] += 1;
+    return Q2_OK;
+  }
   if (use_fused(M, B)) {
     Q2_TRY(fused_layers(M, B, st));  // the residual stream ends in x
   } else {
@@ -933,6 +1021,50 @@ q2_status q2_model_time_kernels(q2_model* M, const int64_t* ids, int B, int step
   DeviceGuard g(M->device);
   cudaStream_t st = as_stream(stream);
   Q2_TRY(check_stream_device(M, st));
+  if (use_persistent(M, B)) {
+    // One kernel per step: per-phase critical-path times from the kernel's
+    // own global-timer stamps (latest end of a phase minus the latest end of
+    // the phase before), and the whole launch by CUDA events.
+    const int L = M->m.n_layers, nph = 5 * L + 1;
+    std::vector<int> saved(M->h_len.begin(), M->h_len.begin() + B);
+    std::vector<double> sum(Q2_K_COUNT, 0.0);
+    std::vector<int> cnt(Q2_K_COUNT, 0);
+    std::vector<unsigned long long> tr((size_t)nph * 4);
+    const int cls[6] = {Q2_K_QKV, Q2_K_ATTN, Q2_K_O, Q2_K_GATE_UP, Q2_K_DOWN, Q2_K_LM_HEAD};
+    cudaEvent_t e0, e1;
+    Q2_CUDA_TRY(cudaEventCreate(&e0));
+    Q2_CUDA_TRY(cudaEventCreate(&e1));
+    for (int r = 0; r < steps; ++r) {
+      Q2_CUDA_TRY(cudaMemcpyAsync(M->d_ids, ids, B * sizeof(int64_t), cudaMemcpyDeviceToDevice, st));
+      Q2_CUDA_TRY(cudaEventRecord(e0, st));
+      Q2_TRY(persistent_step(M, B, true, true, st, true));
+      Q2_CUDA_TRY(cudaEventRecord(e1, st));
+      Q2_CUDA_TRY(cudaStreamSynchronize(st));
+      float ms = 0.f;
+      Q2_CUDA_TRY(cudaEventElapsedTime(&ms, e0, e1));
+      sum[Q2_K_STEP] += ms;
+      Q2_CUDA_TRY(cudaMemcpy(tr.data(), M->d_trace, tr.size() * sizeof(unsigned long long),
+                             cudaMemcpyDeviceToHost));
+      for (int ph = 0; ph < nph; ++ph) {
+        const unsigned long long end = tr[ph * 4 + 0];
+        const unsigned long long prev = ph == 0 ? tr[1] : tr[(ph - 1) * 4 + 0];
+        const int kind = ph == 5 * L ? 5 : ph % 5;
+        sum[cls[kind]] += (double)(end - prev) * 1e-6;  // ns -> ms
+      }
+      Q2_CUDA_TRY(cudaMemcpy(M->d_len, saved.data(), B * sizeof(int), cudaMemcpyHostToDevice));
+    }
+    cudaEventDestroy(e0);
+    cudaEventDestroy(e1);
+    cnt[Q2_K_QKV] = cnt[Q2_K_ATTN] = cnt[Q2_K_O] = cnt[Q2_K_GATE_UP] = cnt[Q2_K_DOWN] = L;
+    cnt[Q2_K_LM_HEAD] = 1;
+    cnt[Q2_K_STEP] = 1;
+    for (int c = 0; c < Q2_K_COUNT; ++c) {
+      per_step[c] = cnt[c];
+      mean_ms[c] = cnt[c] ? (float)(sum[c] / ((double)cnt[c] * steps)) : 0.f;
+    }
+    *kernels_per_step = 1;
+    return Q2_OK;
+  }
   KTiming* t = nullptr;
   auto it = M->timed.find(B);
   if (it == M->timed.end()) {
@@ -1027,6 +1159,31 @@ q2_status q2_model_head(q2_model* M, const void* x, int rows, int64_t* next, flo
   if (logits)
     Q2_CUDA_TRY(cudaMemcpyAsync(logits, M->logits, (size_t)rows * M->m.vocab * sizeof(float),
                                 cudaMemcpyDeviceToDevice, st));
+  return Q2_OK;
+}
+
+q2_status q2_model_set_decode_path(q2_model* M, int path) {
+  clear_error();
+  Q2_CHECK_ARG(M, Q2_ERR_INVALID_ARG, "set_decode_path: NULL model");
+  Q2_CHECK_ARG(path >= Q2_PATH_AUTO && path <= Q2_PATH_GENERIC, Q2_ERR_INVALID_ARG,
+               "set_decode_path: bad path");
+  Q2_CHECK_ARG(path != Q2_PATH_PERSISTENT || M->persistent, Q2_ERR_STATE,
+               "set_decode_path: the persistent kernel does not support this model");
+  Q2_CHECK_ARG(path != Q2_PATH_KERNELS || M->fused, Q2_ERR_STATE,
+               "set_decode_path: the fused kernels do not support this model");
+  if (path != M->path) {
+    DeviceGuard g(M->device);
+    cudaDeviceSynchronize();
+    for (auto& kv : M->graphs) cudaGraphExecDestroy(kv.second);
+    M->graphs.clear();
+    for (auto& kv : M->timed) {
+      if (kv.second->exec) cudaGraphExecDestroy(kv.second->exec);
+      for (cudaEvent_t e : kv.second->ev) cudaEventDestroy(e);
+      delete kv.second;
+    }
+    M->timed.clear();
+  }
+  M->path = path;
   return Q2_OK;
 }
 

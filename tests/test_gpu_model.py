@@ -296,3 +296,60 @@ def test_decode_step_host_matches_device_path(tiny_w):
         n2 = gm2.decode_step(n2)
         dev.append(int(n2[0]))
     assert host == dev
+
+
+# ------------------------------------------------ decode implementations
+
+@pytest.mark.parametrize("B", [1, 3])
+def test_decode_paths_agree_with_each_other_and_the_oracle(mid, B):
+    """The persistent step, the five-kernel fused path and the per-operator
+    path compute the same decode steps (teacher-forced ids, B sequences)."""
+    shape, w = mid
+    lens = [20, 33, 7][:B]
+    prompts = [synth.prompt_ids(shape, n, 40 + b, seq=b) for b, n in enumerate(lens)]
+    feeds = [synth.uniform_ids(B, shape.vocab, 90 + i) for i in range(4)]
+    gm = q2.Model(shape, max_seq=128, max_batch=4)
+    gm.load(w)
+    out = {}
+    for path in ("persistent", "kernels", "generic"):
+        gm.set_decode_path(path)
+        gm.reset_kv()
+        gm.prefill(torch.cat(prompts).cuda(), lens)
+        lg = []
+        for f in feeds:
+            _, l = gm.decode_step(f.cuda(), want_logits=True)
+            lg.append(l.cpu())
+        gm.check_error()
+        out[path] = lg
+    for path in ("persistent", "kernels"):
+        for a, b in zip(out[path], out["generic"]):
+            for r in range(B):
+                assert_bf16_logits(a[r], b[r], f"{path} vs generic, row {r}")
+    # and the first decode step of sequence 0 against the oracle
+    om = oracle.OracleModel(shape, max_seq=128)
+    om.load({k: t.cpu() for k, t in w.items()})
+    om.forward(0, prompts[0])
+    _, ref = om.forward(0, feeds[0][:1])
+    assert_bf16_logits(out["persistent"][0][0], ref, "persistent vs oracle")
+
+
+def test_persistent_step_is_deterministic_and_graph_safe(mid):
+    shape, w = mid
+    gm = q2.Model(shape, max_seq=64, max_batch=2)
+    gm.load(w)
+    gm.set_decode_path("persistent")
+    prompt = synth.prompt_ids(shape, 12, 8).cuda()
+    runs = []
+    for graphs in (True, False, True):
+        gm.reset_kv()
+        gm.set_graphs(graphs)
+        nxt = gm.prefill(torch.cat([prompt, prompt]), [12, 12])
+        lgs = []
+        for _ in range(6):
+            nxt, lg = gm.decode_step(nxt, want_logits=True)
+            lgs.append(lg.clone())
+        runs.append(lgs)
+        gm.check_error()
+    for x, y, z in zip(*runs):
+        assert bits_equal(x, y) and bits_equal(x, z)
+    assert gm.get_seq_len(0) == gm.get_seq_len(1) == 18
