@@ -295,7 +295,8 @@ q2_status q2_model_check_error(q2_model* model, void* stream);
 q2_status q2_model_set_graphs(q2_model* model, int enable);
 
 /* Decode-step implementation for bf16 models at batch <= 4:
- * Q2_PATH_AUTO (default: the fused per-layer kernels where the shapes allow),
+ * Q2_PATH_AUTO (default: the persistent kernel for 2 <= batch <= 4, the fused
+ * per-layer kernels at batch 1, where the shapes allow),
  * Q2_PATH_PERSISTENT (one cooperative launch per step: every CTA streams its
  * share of all weights through one TMA ring while the phases of the step run
  * between grid-wide counters), Q2_PATH_KERNELS (five fused kernels per layer

@@ -19,6 +19,7 @@
 #include "decode.h"
 #include "kernels.h"
 #include "pdecode.h"
+#include <cstdlib>
 #include "tma.h"
 
 using namespace q2;
@@ -84,6 +85,9 @@ struct q2_model {
   bool fused = false;              // bf16 and the fused decode kernels support the shapes
   bool persistent = false;         // ... and the persistent decode kernel does too
   int path = Q2_PATH_AUTO;
+  // Weight stages each CTA of the persistent step pulls into L2 ahead of its
+  // shared-memory ring (Q2_PDECODE_L2_AHEAD overrides; 0 turns it off).
+  int l2_ahead = 16;
   PLayer* d_layers = nullptr;      // device copy of the per-layer weight pointers
   unsigned* d_sync = nullptr;      // persistent step phase counters
   unsigned long long* d_trace = nullptr;  // persistent step phase timestamps [5L + 1][4]
@@ -297,7 +301,10 @@ q2_status run_head(q2_model* M, int r0, int rows, int lrow, cudaStream_t st, boo
 // per layer, norms/RoPE/KV append/SwiGLU/residual adds in the linears'
 // prologues and epilogues, split attention with its combine folded in.
 bool use_persistent(const q2_model* M, int B) {
-  return M->persistent && B >= 1 && B <= kPMaxBatch && M->path == Q2_PATH_PERSISTENT;
+  // AUTO: the persistent step where it is measured faster than the per-layer
+  // kernels (2 <= B <= 4 on B200; at B = 1 the per-layer kernels win).
+  return M->persistent && B >= 1 && B <= kPMaxBatch &&
+         (M->path == Q2_PATH_PERSISTENT || (M->path == Q2_PATH_AUTO && B >= 2));
 }
 bool use_fused(const q2_model* M, int B) {
   return M->fused && B >= 1 && B <= kDecodeMaxBatch && M->path != Q2_PATH_GENERIC;
@@ -324,6 +331,7 @@ q2_status persistent_step(q2_model* M, int B, bool head, bool embed_in, cudaStre
   p.nsplit = decode_splits(M, B);
   p.eps = m.eps;
   p.scale = 1.0f / sqrtf((float)m.head_dim);
+  p.l2_ahead = M->l2_ahead;
   p.embed_in = embed_in ? 1 : 0;
   p.run_head = head ? 1 : 0;
   p.embed = M->embed;
@@ -719,6 +727,10 @@ q2_status q2_model_create(const q2_meta* meta, int device, q2_model** out) {
     M->fused = (vs == Q2_OK) && rows < (1ull << 31);
     M->persistent = M->fused && pdecode_supported(m.hidden, m.intermediate, m.vocab, m.n_heads,
                                                   m.n_kv_heads, m.head_dim, M->qkvd, M->qd);
+    if (const char* env = getenv("Q2_PDECODE_L2_AHEAD")) {
+      const int v = atoi(env);
+      if (v >= 0 && v <= 256) M->l2_ahead = v;
+    }
     clear_error();
   }
   {

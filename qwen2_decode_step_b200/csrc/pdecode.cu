@@ -15,8 +15,11 @@ using bf16 = __nv_bfloat16;
 namespace {
 
 constexpr int kC = kPConsumers;             // consumer warps
-constexpr int kThreads = (kC + 1) * 32;     // + one producer warp
-constexpr int kSlot = 24 * 1024;            // ring slot (largest weight stage)
+constexpr int kThreads = (kC + 2) * 32;     // + the producer and the epilogue warp
+constexpr int kSlot = 8 * (1536 * 2 + 64);  // ring slot: 8 padded rows of K = 1536
+constexpr int kRowPad = 64;                 // bytes between staged rows beyond K (bank spread)
+constexpr int kActPad = 32;                 // bf16 elements of padding per activation row
+constexpr int kEpiRows = 64;                // output rows per CTA with staged epilogue operands
 constexpr int kAT = 64;                     // attention keys per tile
 constexpr int kHD = 128;                    // head dim of this kernel
 constexpr int kTileBytes = kAT * kHD * 2;   // one K (or V) tile
@@ -31,7 +34,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 struct PGeo {
   int ring;          // weight ring slots
   int act_elems;     // per-token activation capacity (max of H, I, qd)
-  size_t o_ring, o_act, o_qs, o_S, o_ml, o_red, o_ami, o_amv, o_bars, o_flag, total;
+  size_t o_ring, o_act, o_qs, o_S, o_ml, o_red, o_bars, o_flag, o_acc, o_epi, total;
 };
 
 __host__ __device__ inline size_t up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -39,35 +42,34 @@ __host__ __device__ inline size_t up(size_t v, size_t a) { return (v + a - 1) / 
 PGeo make_geo(int mt, int act_elems) {
   PGeo g;
   g.act_elems = act_elems;
-  size_t o = 2 * 2 * (size_t)kTileBytes;  // attention K/V tiles, two stages (reused by the O prologue)
-  g.o_ring = o;                           // ring follows (filled below)
-  size_t fixed = up((size_t)mt * act_elems * 2, 16) + kAGMax * kHD * 4 + kAGMax * kAT * 4 +
-                 3 * kAGMax * 4 + kC * 4 * 4 + kC * 4 * 8 + kC * 4 * 4 + 64 * 8 + 64;
-  long long room = (long long)kSmemMax - 1024 - (long long)o - (long long)fixed;
-  int ring = (int)(room / kSlot);
-  if (ring > 8) ring = 8;
-  g.ring = ring;
-  o += (size_t)ring * kSlot;
-  g.o_act = o;
-  o = up(o + (size_t)mt * act_elems * 2, 16);
-  g.o_qs = o;
-  o += kAGMax * kHD * 4;
-  g.o_S = o;
-  o += kAGMax * kAT * 4;
-  g.o_ml = o;
-  o += 3 * kAGMax * 4;
-  g.o_red = o;
-  o += kC * 4 * 4;
-  g.o_ami = up(o, 8);
-  o = g.o_ami + kC * 4 * 8;
-  g.o_amv = o;
-  o += kC * 4 * 4;
-  g.o_bars = up(o, 8);
-  o = g.o_bars + ((size_t)ring + 2) * 8 + (size_t)ring * 4;  // full[ring], abar[2], released[ring]
-  o = up(o, 8);
-  g.o_flag = o;
-  o += 16;
-  g.total = o + 1024;  // slack for aligning the base
+  for (int ring = 8; ring >= 1; --ring) {
+    size_t o = 2 * 2 * (size_t)kTileBytes;  // attention K/V tiles, two stages
+    g.o_ring = o;
+    o += (size_t)ring * kSlot;
+    g.o_act = o;
+    o = up(o + (size_t)mt * (act_elems + kActPad) * 2, 16);
+    g.o_qs = o;
+    o += kAGMax * kHD * 4;
+    g.o_S = o;
+    o += kAGMax * kAT * 4;
+    g.o_ml = o;
+    o += 3 * kAGMax * 4;
+    g.o_red = o;
+    o += kC * 4 * 4;
+    g.o_bars = up(o, 8);
+    // full[ring], empty[ring], posted[ring + 1], epid[ring + 1], abar[2]
+    o = g.o_bars + (2 * (size_t)ring + 2 * (size_t)(ring + 1) + 2) * 8;
+    o = up(o, 8);
+    g.o_flag = o;
+    o += 16;
+    g.o_acc = o;  // per-warp row-group sums [ring + 1][kC][8 rows][4 tokens]
+    o += (size_t)(ring + 1) * kC * 8 * 4 * 4;
+    g.o_epi = o;  // staged epilogue operands: bias, RoPE cos/sin, residual rows
+    o += (size_t)kEpiRows * 4 * (1 + 2 + 4);
+    g.ring = ring;
+    g.total = o + 1024;  // slack for aligning the base
+    if (g.total <= kSmemMax) break;
+  }
   return g;
 }
 
@@ -83,25 +85,26 @@ __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
   return v;
 }
 
+// try_wait that lets the hardware suspend the thread for up to `ns` while the
+// phase is still open (a waiting warp then takes no issue slots).
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
 // mbarrier wait with a deadline; false if it ran out.
 __device__ __forceinline__ bool mwait(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = gtimer();
   for (;;) {
-    for (int i = 0; i < 256; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
-    if (gtimer() - t0 > kDeadlineNs) return false;
-  }
-}
-
-// Wait until a shared-memory counter reaches `target` (deadline-bounded).
-__device__ __forceinline__ bool wait_count(const unsigned* c, unsigned target) {
-  const volatile unsigned* vc = c;
-  if (*vc >= target) return true;
-  const uint64_t t0 = gtimer();
-  for (;;) {
-    for (int i = 0; i < 64; ++i)
-      if (*vc >= target) return true;
+    for (int i = 0; i < 16; ++i)
+      if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
     if (gtimer() - t0 > kDeadlineNs) return false;
   }
 }
@@ -122,37 +125,109 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 
 __device__ __forceinline__ float silu_mul(float gv, float uv) { return uv * (gv / (1.0f + expf(-gv))); }
 
+// c += A . B for one m16n8k16 tile, bf16 operands, fp32 accumulators.  A rows
+// 8..15 are zero: only a0 (row g, k pair 2t) and a2 (row g, k pair 2t + 8) are
+// passed; b0 and b1 are column g's k pairs 2t and 2t + 8.
+__device__ __forceinline__ void mma_bf16_16816(float* c, uint32_t a0, uint32_t a2, uint32_t b0,
+                                               uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+
 __device__ __forceinline__ int swz(int r, int c) {
   return r * 128 + ((((c >> 3) ^ (r & 7)) << 4) | ((c & 7) << 1));
 }
 
 enum { PH_QKV = 0, PH_ATTN = 1, PH_O = 2, PH_GU = 3, PH_DOWN = 4, PH_HEAD = 5 };
 
+// A weight phase streams W [N][K] in stages of R rows x KT columns (kb = K / KT
+// column blocks per group of R rows); each CTA owns the row groups [gb, ge).
 struct WPhase {
   const bf16* w;
-  int N, K, R, rpu, kind;
+  int N, K, R, KT, kb, stride, kind, gb, ge;
 };
+
+// Rows per group: 8, or 4 where that cuts the rows of the busiest CTA by at
+// least an eighth (small N, e.g. the o and down projections).
+__host__ __device__ inline int phase_rows(int N, int G) {
+  const int c8 = (N + 8 * G - 1) / (8 * G) * 8, c4 = (N + 4 * G - 1) / (4 * G) * 4;
+  return 8 * c4 <= 7 * c8 ? 4 : 8;
+}
+
+// Column blocks: the fewest with KT a multiple of 256 whose R padded rows fit a slot.
+__host__ __device__ inline int phase_kblocks(int K, int R) {
+  if (K % 256 != 0) return 0;
+  for (int kb = 1; kb <= K / 256; ++kb)
+    if ((K / 256) % kb == 0 && (size_t)R * ((size_t)(K / kb) * 2 + kRowPad) <= (size_t)kSlot) return kb;
+  return 0;
+}
 
 __device__ __forceinline__ int phase_kind(const PDecode& p, int ph) {
   return ph == 5 * p.L ? PH_HEAD : ph % 5;
 }
 
-__device__ __forceinline__ bool weight_phase(const PDecode& p, int ph, WPhase& wp) {
+__device__ __forceinline__ bool weight_phase(const PDecode& p, int ph, int bid, int G, WPhase& wp) {
   const int kind = phase_kind(p, ph);
   if (kind == PH_ATTN) return false;
   const PLayer* Lw = kind == PH_HEAD ? nullptr : &p.layers[ph / 5];
   switch (kind) {
-    case PH_QKV: wp.w = (const bf16*)Lw->wqkv; wp.N = p.qkvd; wp.K = p.H; wp.rpu = 2; break;
-    case PH_O: wp.w = (const bf16*)Lw->wo; wp.N = p.H; wp.K = p.qd; wp.rpu = 1; break;
-    case PH_GU: wp.w = (const bf16*)Lw->wgu; wp.N = 2 * p.I; wp.K = p.H; wp.rpu = 2; break;
-    case PH_DOWN: wp.w = (const bf16*)Lw->wd; wp.N = p.H; wp.K = p.I; wp.rpu = 1; break;
-    default: wp.w = (const bf16*)p.lm_head; wp.N = p.V; wp.K = p.H; wp.rpu = 1; break;
+    case PH_QKV: wp.w = (const bf16*)Lw->wqkv; wp.N = p.qkvd; wp.K = p.H; break;
+    case PH_O: wp.w = (const bf16*)Lw->wo; wp.N = p.H; wp.K = p.qd; break;
+    case PH_GU: wp.w = (const bf16*)Lw->wgu; wp.N = 2 * p.I; wp.K = p.H; break;
+    case PH_DOWN: wp.w = (const bf16*)Lw->wd; wp.N = p.H; wp.K = p.I; break;
+    default: wp.w = (const bf16*)p.lm_head; wp.N = p.V; wp.K = p.H; break;
   }
-  int r = 8;
-  while (r > wp.rpu && r * wp.K * 2 > kSlot) r >>= 1;
-  wp.R = r;
+  wp.R = phase_rows(wp.N, G);
+  wp.kb = phase_kblocks(wp.K, wp.R);
+  wp.KT = wp.K / wp.kb;
+  wp.stride = wp.KT * 2 + kRowPad;
   wp.kind = kind;
+  const int ng = (wp.N + wp.R - 1) / wp.R;
+  wp.gb = (int)((long long)bid * ng / G);
+  wp.ge = (int)((long long)(bid + 1) * ng / G);
   return true;
+}
+
+// The sequence of weight stages one CTA streams: phase by phase, for each of
+// its row groups the kb column blocks in order (no divisions per stage).
+struct StageIter {
+  WPhase wp;
+  int ph, grp, kblk;
+  __device__ void enter(const PDecode& p, int bid, int G, int nph) {
+    for (; ph < nph; ++ph) {
+      if (!weight_phase(p, ph, bid, G, wp)) continue;
+      grp = wp.gb;
+      kblk = 0;
+      if (wp.gb < wp.ge) return;
+    }
+    grp = 0;
+    wp.ge = 0;
+  }
+  __device__ void begin(const PDecode& p, int bid, int G, int nph) {
+    ph = 0;
+    enter(p, bid, G, nph);
+  }
+  __device__ bool valid() const { return grp < wp.ge; }
+  __device__ void next(const PDecode& p, int bid, int G, int nph) {
+    if (++kblk < wp.kb) return;
+    kblk = 0;
+    if (++grp < wp.ge) return;
+    ++ph;
+    enter(p, bid, G, nph);
+  }
+  __device__ int rows() const { return min(wp.R, wp.N - grp * wp.R); }
+  __device__ uint32_t bytes() const { return (uint32_t)rows() * wp.KT * 2; }
+  // row r of the stage in global memory
+  __device__ const bf16* src(int r) const {
+    return wp.w + (size_t)(grp * wp.R + r) * wp.K + (size_t)kblk * wp.KT;
+  }
+};
+
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 }  // namespace
@@ -173,19 +248,27 @@ __global__ void __launch_bounds__(kThreads, 1) pdecode_kernel(const PDecode p, c
   float* ls = ms + kAGMax;
   float* al = ls + kAGMax;
   float* red = reinterpret_cast<float*>(smem + g.o_red);
-  long long* ami = reinterpret_cast<long long*>(smem + g.o_ami);
-  float* amv = reinterpret_cast<float*>(smem + g.o_amv);
+  // Weight ring: full[slot] completes when a stage's bytes have landed,
+  // empty[slot] when all kC consumer warps have passed the stage.  Every
+  // consumer warp passes every stage, in order, computing only its own units,
+  // so no waiter is ever more than one phase away from the barrier it waits
+  // on and every parity wait is unambiguous.
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + g.o_bars);
-  uint64_t* abar = full + g.ring;
-  // released[slot]: cumulative count of consumer releases of that slot, kC per
-  // use.  A cumulative count (rather than a parity wait on an mbarrier) lets a
-  // consumer that runs several uses ahead of another warp tell exactly which
-  // use of the slot is resident.
-  unsigned* released = reinterpret_cast<unsigned*>(abar + 2);
+  uint64_t* empty = full + g.ring;
+  // Row-group accumulators: posted[a] completes when all kC consumer warps
+  // have written their partial sums of the group on accumulator a, epid[a]
+  // when the epilogue warp has finished that group.
+  uint64_t* posted = empty + g.ring;
+  uint64_t* epid = posted + g.ring + 1;
+  uint64_t* abar = epid + g.ring + 1;
   int* s_flags = reinterpret_cast<int*>(smem + g.o_flag);
   int& s_flag = s_flags[0];
   int& s_last_merge = s_flags[1];
   int& s_pre = s_flags[2];  // attention tiles of this CTA's first item already in flight
+  float* acc_s = reinterpret_cast<float*>(smem + g.o_acc);        // [ring + 1][kC][8][4]
+  float* e_bias = reinterpret_cast<float*>(smem + g.o_epi);       // [kEpiRows]
+  float2* e_cs = reinterpret_cast<float2*>(e_bias + kEpiRows);    // [kEpiRows / 2][4]
+  float* e_x = reinterpret_cast<float*>(e_cs + kEpiRows / 2 * 4);  // [kEpiRows][4]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x, bid = blockIdx.x;
@@ -195,7 +278,11 @@ __global__ void __launch_bounds__(kThreads, 1) pdecode_kernel(const PDecode p, c
   if (tid == 0) {
     for (int i = 0; i < RING; ++i) {
       mbar_init(&full[i], 1);
-      released[i] = 0;
+      mbar_init(&empty[i], kC);
+    }
+    for (int i = 0; i <= RING; ++i) {
+      mbar_init(&posted[i], kC);
+      mbar_init(&epid[i], 1);
     }
     mbar_init(&abar[0], 1);
     mbar_init(&abar[1], 1);
@@ -203,30 +290,182 @@ __global__ void __launch_bounds__(kThreads, 1) pdecode_kernel(const PDecode p, c
   }
   __syncthreads();
 
+  const int NACC = RING + 1;  // row-group accumulators (see the producer)
+  const unsigned ARRIVALS = 2u * (unsigned)G;  // per phase: consumers and producer of every CTA
+
+  // The last arrival of the last phase wraps up the step: the step's token
+  // per sequence (argmax over the CTAs' partials) and the lengths.
+  auto wrap_up = [&](int t) {  // t: thread index within the caller's group
+    __threadfence();
+    if (t < p.B) {
+      if (p.run_head) {
+        float bv = -INFINITY;
+        long long bi = LLONG_MAX;
+        for (int b = 0; b < G; ++b) {
+          const float v = __ldcg(p.am_val + b * 4 + t);
+          const long long i = __ldcg(reinterpret_cast<const long long*>(p.am_idx) + b * 4 + t);
+          if (am_better(v, i, bv, bi)) {
+            bv = v;
+            bi = i;
+          }
+        }
+        p.next[t] = bi;
+      }
+      p.lens[t] += 1;
+    }
+  };
+
   // ================================================================ producer
+  // Lane 0 waits for a free slot and arms its barrier; lanes r < rows then
+  // issue the copy of row r, and lane 31 pulls a later stage into L2.  Before
+  // the first stage of a group it also waits until the epilogue warp is done
+  // with the group that last used the group's accumulator.
   if (warp == kC) {
-    if (lane == 0) {
-      const uint64_t pol = policy_evict_first();
-      long long gs = 0;
-      for (int ph = 0; ph < nph; ++ph) {
-        WPhase wp;
-        if (!weight_phase(p, ph, wp)) continue;
-        const int Sn = (wp.N + wp.R - 1) / wp.R;
-        const int sb = (int)((long long)bid * Sn / G), se = (int)((long long)(bid + 1) * Sn / G);
-        for (int s = sb; s < se; ++s, ++gs) {
-          const int slot = (int)(gs % RING);
-          const long long k = gs / RING;
-          // Reuse of a slot waits for every consumer release of its previous
-          // use (their reads of the slot are complete before they release it).
-          if (k >= 1 && !wait_count(&released[slot], (unsigned)(k * kC))) atomicOr(p.err, 2);
-          const int rows = min(wp.R, wp.N - s * wp.R);
-          const uint32_t bytes = (uint32_t)rows * wp.K * 2;
-          mbar_arrive_expect_tx(&full[slot], bytes);
-          bulk_g2s_evict_first(ring + (size_t)slot * kSlot, wp.w + (size_t)s * wp.R * wp.K, bytes,
-                               &full[slot], pol);
+    const uint64_t pol = policy_evict_first();
+    // `ahead` runs p.l2_ahead stages in front of the ring and pulls them into
+    // L2 (a group's rows are contiguous in W: all of them when its first
+    // column block comes up), so HBM keeps streaming while the ring is full
+    // (during the grid barriers and the attention phase).
+    StageIter cur, ahead;
+    cur.begin(p, bid, G, nph);
+    ahead.begin(p, bid, G, nph);
+    auto prefetch = [&](const StageIter& a) {
+      if (lane == 31 && a.kblk == 0) bulk_prefetch_l2(a.src(0), (uint32_t)a.rows() * a.wp.K * 2);
+    };
+    for (int i = 0; i < p.l2_ahead && ahead.valid(); ++i, ahead.next(p, bid, G, nph)) prefetch(ahead);
+    int slot = 0;
+    uint32_t par = 0;
+    int acc_i = 0;          // accumulator of the next group
+    long long groups = 0;   // groups started
+    for (long long gs = 0; cur.valid(); ++gs, cur.next(p, bid, G, nph)) {
+      if (lane == 0) {
+        // Reuse of a slot waits until every consumer warp has passed its
+        // previous use (their reads of the slot are complete by then).
+        if (gs >= RING && !mwait(&empty[slot], par ^ 1u)) atomicOr(p.err, 2);
+        if (cur.kblk == 0) {
+          if (groups >= NACC && !mwait(&epid[acc_i], (uint32_t)((groups / NACC - 1) & 1)))
+            atomicOr(p.err, 2);
+          ++groups;
+          acc_i = acc_i + 1 == NACC ? 0 : acc_i + 1;
+        }
+        mbar_arrive_expect_tx(&full[slot], cur.bytes());
+      }
+      __syncwarp();
+      if (lane < cur.rows())  // one copy per row: rows land wp.stride bytes apart
+        bulk_g2s_evict_first(ring + (size_t)slot * kSlot + (size_t)lane * cur.wp.stride, cur.src(lane),
+                             (uint32_t)cur.wp.KT * 2, &full[slot], pol);
+      if (ahead.valid()) {
+        prefetch(ahead);
+        ahead.next(p, bid, G, nph);
+      }
+      if (++slot == RING) {
+        slot = 0;
+        par ^= 1u;
+      }
+    }
+    return;
+  }
+
+  // ========================================================= epilogue warp
+  // Finishes every row group once its partial sums are posted (lane (r, m):
+  // row r, token m), and signals each phase's end to the grid once that
+  // phase's last group is written.
+  if (warp == kC + 1) {
+    StageIter epi;
+    epi.begin(p, bid, G, nph);
+    const int r = lane >> 2, m = lane & 3;
+    float best_v = -INFINITY;  // lm_head argmax of token m over this lane's rows
+    long long best_i = LLONG_MAX;
+    int arrived = 0;  // phases [0, arrived) signalled
+    auto signal_until = [&](int ph_end) {
+      for (; arrived < ph_end; ++arrived) {
+        if (phase_kind(p, arrived) == PH_HEAD) {  // this CTA's argmax partial per token
+#pragma unroll
+          for (int o = 4; o < 32; o <<= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, best_v, o);
+            const long long oi = __shfl_xor_sync(0xffffffffu, best_i, o);
+            if (am_better(ov, oi, best_v, best_i)) {
+              best_v = ov;
+              best_i = oi;
+            }
+          }
+          if (lane < 4) {
+            p.am_val[bid * 4 + lane] = best_v;
+            p.am_idx[bid * 4 + lane] = best_i;
+          }
+        }
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) {
+          if (p.trace) atomicMax(&p.trace[arrived * 4 + 0], (unsigned long long)gtimer());
+          last = atom_add_release(&p.sync[arrived], 1u) == ARRIVALS - 1 && arrived == nph - 1;
+        }
+        if (__shfl_sync(0xffffffffu, last, 0)) wrap_up(lane);
+      }
+    };
+    signal_until(epi.valid() ? epi.ph : nph);
+    int acc_i = 0;
+    long long groups = 0;
+    for (; epi.valid(); epi.next(p, bid, G, nph), signal_until(epi.valid() ? epi.ph : nph)) {
+      const WPhase& wp = epi.wp;
+      if (epi.kblk != wp.kb - 1) continue;  // the group ends at its last column block
+      const int ai = acc_i;
+      acc_i = acc_i + 1 == NACC ? 0 : acc_i + 1;
+      if (lane == 0 && !mwait(&posted[ai], (uint32_t)((groups / NACC) & 1))) atomicOr(p.err, 2);
+      ++groups;
+      __syncwarp();
+      const float* acc = acc_s + ai * (kC * 32);
+      float v = 0.f;
+#pragma unroll
+      for (int w = 0; w < kC; ++w) v += acc[w * 32 + r * 4 + m];
+      const float vn = __shfl_down_sync(0xffffffffu, v, 4);  // row r + 1, token m
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&epid[ai]);  // the accumulator is read
+      const int R = wp.R, rows = epi.rows();
+      const int n = epi.grp * R + r, i = n - wp.gb * R;  // output row, staged operand index
+      if (r >= rows || m >= p.B) continue;
+      const int kind = wp.kind, l = epi.ph / 5;
+      if (kind == PH_O || kind == PH_DOWN) {
+        const bf16 xn = from_f<bf16>(e_x[i * 4 + m] + round_st<bf16>(v));
+        reinterpret_cast<bf16*>(p.x)[(size_t)m * p.H + n] = xn;
+        e_x[i * 4 + m] = __bfloat162float(xn);
+      } else if (kind == PH_GU) {
+        if ((r & 1) == 0) {
+          const float gv = round_st<bf16>(v), uv = round_st<bf16>(vn);
+          reinterpret_cast<bf16*>(p.s)[(size_t)m * p.I + (n >> 1)] = from_f<bf16>(silu_mul(gv, uv));
+        }
+      } else if (kind == PH_QKV) {
+        if ((r & 1) == 0) {
+          const int hs = n / p.hd, j = (n % p.hd) >> 1, half = p.hd >> 1;
+          const float va = round_st<bf16>(v + e_bias[i]);
+          const float vb = round_st<bf16>(vn + e_bias[i + 1]);
+          const size_t loff = (size_t)l * p.kv_layer_stride + (size_t)m * p.kv_seq_stride;
+          const int pos = p.lens[m];
+          if (hs < p.nh + p.nkv) {
+            const float2 cs = e_cs[(i >> 1) * 4 + m];
+            const bf16 ra = from_f<bf16>(va * cs.x - vb * cs.y);
+            const bf16 rb = from_f<bf16>(vb * cs.x + va * cs.y);
+            bf16* dst = hs < p.nh ? reinterpret_cast<bf16*>(p.qb) + (size_t)m * p.qd + (size_t)hs * p.hd
+                                  : reinterpret_cast<bf16*>(p.kc) + loff +
+                                        ((size_t)(hs - p.nh) * p.max_seq + pos) * p.hd;
+            dst[j] = ra;
+            dst[j + half] = rb;
+          } else {
+            bf16* vr = reinterpret_cast<bf16*>(p.vc) + loff +
+                       ((size_t)(hs - p.nh - p.nkv) * p.max_seq + pos) * p.hd;
+            vr[j] = from_f<bf16>(va);
+            vr[j + half] = from_f<bf16>(vb);
+          }
+        }
+      } else {  // PH_HEAD
+        p.logits[(size_t)m * p.V + n] = v;
+        if (am_better(v, n, best_v, best_i)) {
+          best_v = v;
+          best_i = n;
         }
       }
     }
+    signal_until(nph);
     return;
   }
 
@@ -234,11 +473,11 @@ __global__ void __launch_bounds__(kThreads, 1) pdecode_kernel(const PDecode p, c
   const int ct = tid;
   const int G_q = p.nh / p.nkv;
   long long gs = 0;  // weight stages consumed so far (same sequence as the producer's)
+  int r_slot = 0;    // ring slot and parity of the next stage
+  uint32_t r_par = 0;
+  int a_slot = 0;    // row-group accumulator of the next group
   int ac = 0;        // attention tile loads issued so far
   const bf16* X = reinterpret_cast<const bf16*>(p.x);
-  // Sequence lengths only change at the very end of the step: lane m keeps
-  // token m's position.
-  const int my_pos = lane < p.B ? p.lens[lane] : 0;
   // TMA load of K/V tile t of (layer l, sequence b, kv head gq) into
   // attention buffer stage li & 1 (issued by one thread).
   auto tile_issue = [&](int l, int b, int gq, int t, int li) {
@@ -272,8 +511,6 @@ __global__ void __launch_bounds__(kThreads, 1) pdecode_kernel(const PDecode p, c
     return a;
   };
   if (ct == 0) s_pre = 0;
-  float best_v = -INFINITY;
-  long long best_i = LLONG_MAX;
 
   // act[m][0..K) = rmsnorm(src[m]) * nw, one rounding (src rows of stride K).
   auto norm_prologue = [&](const bf16* const* src_rows, const bf16* nw, int K) {
@@ -315,164 +552,125 @@ __global__ void __launch_bounds__(kThreads, 1) pdecode_kernel(const PDecode p, c
           unpack16<bf16>(__ldcg(reinterpret_cast<const uint4*>(src_rows[m] + k)), f);
 #pragma unroll
           for (int e = 0; e < 8; ++e) f[e] = f[e] * inv[m] * wf[e];
-          *reinterpret_cast<uint4*>(act + (size_t)m * K + k) = pack16<bf16>(f);
+          *reinterpret_cast<uint4*>(act + (size_t)m * (K + kActPad) + k) = pack16<bf16>(f);
         }
       }
     }
     csync();
   };
 
-  // One weight phase: stream this CTA's stages, run the epilogue per unit.
-  auto gemv_phase = [&](const WPhase& wp, int l) {
-    const int Sn = (wp.N + wp.R - 1) / wp.R;
-    const int sb = (int)((long long)bid * Sn / G), se = (int)((long long)(bid + 1) * Sn / G);
-    const int ns = se - sb;
-    const int units = wp.R / wp.rpu;
-    const uint32_t arrive_cnt = (uint32_t)(kC / units);
-    const int K = wp.K, nch = K / 8;
-    // MT == 1 and K == 1536: the activation stays in registers (6 chunks per lane).
-    constexpr int NXR = MT == 1 ? 6 : 1;
-    const bool regs = (MT == 1) && (K == 6 * 256);
-    float xr[NXR][8];
-    if (regs) {
+  // One weight phase on the tensor cores (mma.sync m16n8k16, bf16 operands,
+  // fp32 accumulation).  M is the token (A rows g < B; the rest are zero), N
+  // the R rows of a stage, K this warp's eighth of the stage's columns.  Lane
+  // (g = lane / 4, t = lane % 4) loads 16 bytes of weight row g and 16 bytes of
+  // token g's activation at the same columns: since a dot product may sum its
+  // terms in any order, those eight columns feed two MMAs directly (one column
+  // permutation shared by both operands).  Each warp keeps its partial sums
+  // of the group in its own slice of the group's accumulator (summing its kb
+  // column blocks in order); the last of the kC * kb contributions runs the
+  // epilogue, lane (r, m) adding the kC slices of row r, token m in warp
+  // order -- a fixed summation order, so every step is bit-reproducible.
+  auto gemv_phase = [&](const WPhase& wp) {
+    const int K = wp.K, KT = wp.KT, kb = wp.kb, R = wp.R;
+    const int ns = (wp.ge - wp.gb) * kb;
+    const int kw = KT / kC;  // columns per warp, a multiple of 32
+    const int g8 = lane >> 2, t4 = lane & 3;
+    const bool act_ok = g8 < p.B;
+    const bf16* act_row = act + (size_t)g8 * (K + kActPad) + warp * kw + 8 * t4;
+    int grp = wp.gb, kblk = -1;
+    for (int t = 0; t < ns; ++t) {
+      const int slot = r_slot;
+      const uint32_t par = r_par;
+      if (++r_slot == RING) {
+        r_slot = 0;
+        r_par ^= 1u;
+      }
+      if (++kblk == kb) {
+        kblk = 0;
+        ++grp;
+      }
+      const int ai = a_slot;
+      if (kblk == kb - 1) a_slot = a_slot + 1 == NACC ? 0 : a_slot + 1;
+      const int rows = min(R, wp.N - grp * R);
+      if (!mwait(&full[slot], par) && lane == 0) atomicOr(p.err, 2);
+      // four independent accumulator chains, summed in a fixed order
+      float c[4][4];
 #pragma unroll
-      for (int i = 0; i < NXR; ++i) unpack16<bf16>(reinterpret_cast<const uint4*>(act)[lane + 32 * i], xr[i]);
-    }
-    for (int item = warp; item < ns * units; item += kC) {
-      const int ls_ = item / units, u = item % units;
-      const long long gsi = gs + ls_;
-      const int slot = (int)(gsi % RING);
-      const long long k = gsi / RING;
-      // Every earlier use of the slot is released (so use k is the one the
-      // producer fills next, and the full barrier's parity is unambiguous).
-      if (k >= 1 && !wait_count(&released[slot], (unsigned)(k * kC)) && lane == 0) atomicOr(p.err, 2);
-      if (!mwait(&full[slot], (uint32_t)(k & 1)) && lane == 0) atomicOr(p.err, 2);
-      const uint8_t* stg = ring + (size_t)slot * kSlot;
-      const int s = sb + ls_;
-      const int row0 = s * wp.R;
-      const int rows = min(wp.R, wp.N - row0);
-      // Operands of the epilogue, loaded before the dot product so that their
-      // latency overlaps it (lane m < B works for token m).
-      const int n0e = row0 + u * wp.rpu;
-      float e_b0 = 0.f, e_b1 = 0.f, e_x = 0.f;
-      float2 e_cs = make_float2(1.f, 0.f);
-      if (lane < p.B && n0e < wp.N) {
-        if (wp.kind == PH_QKV) {
-          const bf16* bias = reinterpret_cast<const bf16*>(p.layers[l].bqkv);
-          e_b0 = to_f(bias[n0e]);
-          e_b1 = to_f(bias[n0e + 1]);
-          const int hs = n0e / p.hd;
-          if (hs < p.nh + p.nkv) e_cs = p.rope[(size_t)my_pos * (p.hd >> 1) + ((n0e % p.hd) >> 1)];
-        } else if (wp.kind == PH_O || wp.kind == PH_DOWN) {
-          e_x = __bfloat162float(
-              __ldcg(reinterpret_cast<const __nv_bfloat16*>(p.x) + (size_t)lane * p.H + n0e));
+      for (int a = 0; a < 4; ++a) c[a][0] = c[a][1] = c[a][2] = c[a][3] = 0.f;
+      {
+        const uint8_t* wr = ring + (size_t)slot * kSlot + (size_t)g8 * wp.stride +
+                            (size_t)(warp * kw + 8 * t4) * 2;
+        const bf16* ar = act_row + (size_t)kblk * KT;
+        const bool wok = g8 < rows;
+        const uint4 z = make_uint4(0, 0, 0, 0);
+        if (kw == 192) {  // K = 1536 in one block: all loads first, then the MMAs
+          uint4 wv[6], av[6];
+#pragma unroll
+          for (int i = 0; i < 6; ++i) wv[i] = wok ? *reinterpret_cast<const uint4*>(wr + 64 * i) : z;
+#pragma unroll
+          for (int i = 0; i < 6; ++i) av[i] = act_ok ? *reinterpret_cast<const uint4*>(ar + 32 * i) : z;
+#pragma unroll
+          for (int i = 0; i < 6; ++i) {
+            mma_bf16_16816(c[(i & 1) * 2], av[i].x, av[i].y, wv[i].x, wv[i].y);
+            mma_bf16_16816(c[(i & 1) * 2 + 1], av[i].z, av[i].w, wv[i].z, wv[i].w);
+          }
+        } else {
+          const int nk = kw / 32;
+#pragma unroll 2
+          for (int i = 0; i < nk; i += 2) {
+            const bool two = i + 1 < nk;
+            const uint4 wv0 = wok ? *reinterpret_cast<const uint4*>(wr + 64 * i) : z;
+            const uint4 av0 = act_ok ? *reinterpret_cast<const uint4*>(ar + 32 * i) : z;
+            const uint4 wv1 = wok && two ? *reinterpret_cast<const uint4*>(wr + 64 * i + 64) : z;
+            const uint4 av1 = act_ok && two ? *reinterpret_cast<const uint4*>(ar + 32 * i + 32) : z;
+            mma_bf16_16816(c[0], av0.x, av0.y, wv0.x, wv0.y);
+            mma_bf16_16816(c[1], av0.z, av0.w, wv0.z, wv0.w);
+            mma_bf16_16816(c[2], av1.x, av1.y, wv1.x, wv1.y);
+            mma_bf16_16816(c[3], av1.z, av1.w, wv1.z, wv1.w);
+          }
         }
       }
-      float y[2][MT];
-#pragma unroll
-      for (int r = 0; r < 2; ++r)
-#pragma unroll
-        for (int m = 0; m < MT; ++m) y[r][m] = 0.f;
-#pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        if (r >= wp.rpu) break;
-        const int rr = u * wp.rpu + r;
-        if (rr >= rows) break;
-        const uint4* wrow = reinterpret_cast<const uint4*>(stg + (size_t)rr * K * 2);
-        if (regs) {
-          float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-          for (int i = 0; i < NXR; ++i) {
-            float wf[8];
-            unpack16<bf16>(wrow[lane + 32 * i], wf);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) acc[e & 3] = fmaf(wf[e], xr[i][e], acc[e & 3]);
-          }
-          y[r][0] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-        } else {
-          float acc[MT][2];
-#pragma unroll
-          for (int m = 0; m < MT; ++m) acc[m][0] = acc[m][1] = 0.f;
-#pragma unroll 4
-          for (int c = lane; c < nch; c += 32) {
-            float wf[8];
-            unpack16<bf16>(wrow[c], wf);
-#pragma unroll
-            for (int m = 0; m < MT; ++m) {
-              if (m < p.B) {
-                float xf[8];
-                unpack16<bf16>(reinterpret_cast<const uint4*>(act + (size_t)m * K)[c], xf);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) acc[m][e & 1] = fmaf(wf[e], xf[e], acc[m][e & 1]);
-              }
-            }
-          }
-#pragma unroll
-          for (int m = 0; m < MT; ++m) y[r][m] = acc[m][0] + acc[m][1];
-        }
+      // lane (g, t): token g's partial sums of rows 2t and 2t + 1
+      float* acc = acc_s + ai * (kC * 32);
+      if (act_ok && 2 * t4 < R) {
+        float* mine = acc + warp * 32 + (2 * t4) * 4 + g8;
+        const float s0 = (c[0][0] + c[1][0]) + (c[2][0] + c[3][0]);
+        const float s1 = (c[0][1] + c[1][1]) + (c[2][1] + c[3][1]);
+        mine[0] = kblk == 0 ? s0 : mine[0] + s0;
+        mine[4] = kblk == 0 ? s1 : mine[4] + s1;
       }
       __syncwarp();
       if (lane == 0) {
-        __threadfence_block();
-        atomicAdd(&released[slot], arrive_cnt);
-      }
-#pragma unroll
-      for (int r = 0; r < 2; ++r)
-#pragma unroll
-        for (int m = 0; m < MT; ++m) y[r][m] = warp_sum(y[r][m]);
-
-      const int m = lane;
-      if (m < p.B && m < MT) {
-        float y0 = 0.f, y1 = 0.f;
-#pragma unroll
-        for (int mm = 0; mm < MT; ++mm)
-          if (mm == m) {
-            y0 = y[0][mm];
-            y1 = y[1][mm];
-          }
-        const int n0 = n0e;
-        if (wp.kind == PH_O || wp.kind == PH_DOWN) {
-          if (n0 < wp.N)
-            reinterpret_cast<bf16*>(p.x)[(size_t)m * p.H + n0] = from_f<bf16>(e_x + round_st<bf16>(y0));
-        } else if (wp.kind == PH_GU) {
-          if (n0 + 1 < wp.N) {
-            const float gv = round_st<bf16>(y0), uv = round_st<bf16>(y1);
-            reinterpret_cast<bf16*>(p.s)[(size_t)m * p.I + (n0 >> 1)] = from_f<bf16>(silu_mul(gv, uv));
-          }
-        } else if (wp.kind == PH_QKV) {
-          if (n0 + 1 < wp.N) {
-            const int hs = n0 / p.hd, j = (n0 % p.hd) >> 1, half = p.hd >> 1;
-            const float va = round_st<bf16>(y0 + e_b0);
-            const float vb = round_st<bf16>(y1 + e_b1);
-            const int pos = my_pos;
-            const size_t loff = (size_t)l * p.kv_layer_stride + (size_t)m * p.kv_seq_stride;
-            if (hs < p.nh + p.nkv) {
-              const bf16 ra = from_f<bf16>(va * e_cs.x - vb * e_cs.y);
-              const bf16 rb = from_f<bf16>(vb * e_cs.x + va * e_cs.y);
-              bf16* dst = hs < p.nh ? reinterpret_cast<bf16*>(p.qb) + (size_t)m * p.qd + (size_t)hs * p.hd
-                                    : reinterpret_cast<bf16*>(p.kc) + loff +
-                                          ((size_t)(hs - p.nh) * p.max_seq + pos) * p.hd;
-              dst[j] = ra;
-              dst[j + half] = rb;
-            } else {
-              bf16* vr = reinterpret_cast<bf16*>(p.vc) + loff +
-                         ((size_t)(hs - p.nh - p.nkv) * p.max_seq + pos) * p.hd;
-              vr[j] = from_f<bf16>(va);
-              vr[j + half] = from_f<bf16>(vb);
-            }
-          }
-        } else {  // PH_HEAD
-          if (n0 < wp.N) {
-            p.logits[(size_t)m * p.V + n0] = y0;
-            if (am_better(y0, n0, best_v, best_i)) {
-              best_v = y0;
-              best_i = n0;
-            }
-          }
-        }
+        mbar_arrive(&empty[slot]);
+        // the release orders this warp's partial sums before the epilogue
+        // warp's reads
+        if (kblk == kb - 1) mbar_arrive(&posted[ai]);
       }
     }
     gs += ns;
+  };
+
+  // Epilogue operands of this CTA's rows, staged in shared memory (visible
+  // after the next consumer barrier): q/k/v biases and the RoPE cos/sin of
+  // each pair for each token; the residual rows for the o and down phases
+  // (afterwards kept current by this CTA's own epilogues, as the o and down
+  // phases split their rows alike).
+  auto stage_qkv = [&](const WPhase& wp, int l, bool rope_too) {
+    const int row_lo = wp.gb * wp.R, nrows = min(wp.ge * wp.R, wp.N) - row_lo;
+    const bf16* bias = reinterpret_cast<const bf16*>(p.layers[l].bqkv);
+    for (int idx = ct; idx < nrows * 4; idx += kC * 32) {
+      const int i = idx >> 2, m = idx & 3, n = row_lo + i;
+      if (m == 0) e_bias[i] = to_f(bias[n]);
+      if (rope_too && (i & 1) == 0 && m < p.B && n / p.hd < p.nh + p.nkv)
+        e_cs[(i >> 1) * 4 + m] = p.rope[(size_t)p.lens[m] * (p.hd >> 1) + ((n % p.hd) >> 1)];
+    }
+  };
+  auto stage_x = [&](const WPhase& wp) {
+    const int row_lo = wp.gb * wp.R, nrows = min(wp.ge * wp.R, wp.N) - row_lo;
+    for (int idx = ct; idx < nrows * 4; idx += kC * 32) {
+      const int i = idx >> 2, m = idx & 3;
+      if (m < p.B) e_x[i * 4 + m] = __bfloat162float(__ldcg(X + (size_t)m * p.H + row_lo + i));
+    }
   };
 
   for (int ph = 0; ph < nph; ++ph) {
@@ -482,7 +680,7 @@ __global__ void __launch_bounds__(kThreads, 1) pdecode_kernel(const PDecode p, c
     if (ph > 0) {
       if (ct == 0) {
         const uint64_t t0 = gtimer();
-        while (ld_acquire(&p.sync[ph - 1]) < (unsigned)G) {
+        while (ld_acquire(&p.sync[ph - 1]) < ARRIVALS) {
           if (gtimer() - t0 > kDeadlineNs) {
             atomicOr(p.err, 2);
             break;
@@ -541,10 +739,11 @@ __global__ void __launch_bounds__(kThreads, 1) pdecode_kernel(const PDecode p, c
                     *reinterpret_cast<const uint4*>(rows_[m] + k);
         }
       }
-      norm_prologue(rows_, reinterpret_cast<const bf16*>(p.layers[l].in_norm), p.H);
       WPhase wp;
-      weight_phase(p, ph, wp);
-      gemv_phase(wp, l);
+      weight_phase(p, ph, bid, G, wp);
+      stage_qkv(wp, l, l == 0);  // RoPE cos/sin depend on the positions only
+      norm_prologue(rows_, reinterpret_cast<const bf16*>(p.layers[l].in_norm), p.H);
+      gemv_phase(wp);
     } else if (kind == PH_ATTN) {
       const int items = p.B * p.nkv * p.nsplit;
       for (int item = bid; item < items; item += G) {
@@ -713,62 +912,46 @@ __global__ void __launch_bounds__(kThreads, 1) pdecode_kernel(const PDecode p, c
         csync();
       }
     } else if (kind == PH_O) {
+      WPhase wp;
+      weight_phase(p, ph, bid, G, wp);
+      if (l == 0) stage_x(wp);
       const bf16* A = reinterpret_cast<const bf16*>(p.att);
       for (int k = ct * 8; k < p.qd; k += kC * 32 * 8)
 #pragma unroll
         for (int m = 0; m < MT; ++m)
           if (m < p.B)
-            *reinterpret_cast<uint4*>(act + (size_t)m * p.qd + k) =
+            *reinterpret_cast<uint4*>(act + (size_t)m * (p.qd + kActPad) + k) =
                 __ldcg(reinterpret_cast<const uint4*>(A + (size_t)m * p.qd + k));
       csync();
-      WPhase wp;
-      weight_phase(p, ph, wp);
-      gemv_phase(wp, l);
+      gemv_phase(wp);
     } else if (kind == PH_GU) {
       const bf16* rows_[MT];
 #pragma unroll
       for (int m = 0; m < MT; ++m) rows_[m] = X + (size_t)m * p.H;
       norm_prologue(rows_, reinterpret_cast<const bf16*>(p.layers[l].post_norm), p.H);
       WPhase wp;
-      weight_phase(p, ph, wp);
-      gemv_phase(wp, l);
+      weight_phase(p, ph, bid, G, wp);
+      gemv_phase(wp);
     } else if (kind == PH_DOWN) {
       const bf16* Sv = reinterpret_cast<const bf16*>(p.s);
       for (int k = ct * 8; k < p.I; k += kC * 32 * 8)
 #pragma unroll
         for (int m = 0; m < MT; ++m)
           if (m < p.B)
-            *reinterpret_cast<uint4*>(act + (size_t)m * p.I + k) =
+            *reinterpret_cast<uint4*>(act + (size_t)m * (p.I + kActPad) + k) =
                 __ldcg(reinterpret_cast<const uint4*>(Sv + (size_t)m * p.I + k));
       csync();
       WPhase wp;
-      weight_phase(p, ph, wp);
-      gemv_phase(wp, l);
+      weight_phase(p, ph, bid, G, wp);
+      gemv_phase(wp);
     } else {  // PH_HEAD
       const bf16* rows_[MT];
 #pragma unroll
       for (int m = 0; m < MT; ++m) rows_[m] = X + (size_t)m * p.H;
       norm_prologue(rows_, reinterpret_cast<const bf16*>(p.final_norm), p.H);
       WPhase wp;
-      weight_phase(p, ph, wp);
-      gemv_phase(wp, l);
-      // this CTA's argmax partial per token
-      if (lane < MT) {
-        ami[warp * 4 + lane] = best_i;
-        amv[warp * 4 + lane] = best_v;
-      }
-      csync();
-      if (ct < p.B) {
-        float bv = -INFINITY;
-        long long bi = LLONG_MAX;
-        for (int w = 0; w < kC; ++w)
-          if (am_better(amv[w * 4 + ct], ami[w * 4 + ct], bv, bi)) {
-            bv = amv[w * 4 + ct];
-            bi = ami[w * 4 + ct];
-          }
-        p.am_val[bid * 4 + ct] = bv;
-        p.am_idx[bid * 4 + ct] = bi;
-      }
+      weight_phase(p, ph, bid, G, wp);
+      gemv_phase(wp);
     }
 
     // ---- this CTA is done with the phase
@@ -782,7 +965,7 @@ __global__ void __launch_bounds__(kThreads, 1) pdecode_kernel(const PDecode p, c
       }
       // release: this CTA's writes of the phase (ordered before by the CTA
       // barrier) are visible to whoever acquires the counter
-      s_flag = (atom_add_release(&p.sync[ph], 1u) == (unsigned)G - 1);
+      s_flag = atom_add_release(&p.sync[ph], 1u) == ARRIVALS - 1 && ph == nph - 1;
     }
     csync();
   }
@@ -796,34 +979,17 @@ __global__ void __launch_bounds__(kThreads, 1) pdecode_kernel(const PDecode p, c
       if (ac > st) mwait(&abar[st], (uint32_t)(((ac - 1 - st) / 2) & 1));
   }
 
-  // ---- the last CTA to finish the last phase wraps up the step
-  if (s_flag) {
-    __threadfence();
-    if (ct < p.B) {
-      if (p.run_head) {
-        float bv = -INFINITY;
-        long long bi = LLONG_MAX;
-        for (int b = 0; b < G; ++b) {
-          const float v = __ldcg(p.am_val + b * 4 + ct);
-          const long long i = __ldcg(reinterpret_cast<const long long*>(p.am_idx) + b * 4 + ct);
-          if (am_better(v, i, bv, bi)) {
-            bv = v;
-            bi = i;
-          }
-        }
-        p.next[ct] = bi;
-      }
-      p.lens[ct] += 1;
-    }
-  }
+  // ---- the last arrival of the last phase wraps up the step
+  if (s_flag) wrap_up(ct);
 }
 
 // ======================================================================
 bool pdecode_supported(int H, int I, int V, int nh, int nkv, int hd, int qkvd, int qd) {
   if (hd != kHD || nkv <= 0 || nh % nkv != 0 || nh / nkv > kAGMax || nh > kNHMax) return false;
-  if (H % 8 || I % 8 || qd % 8 || qkvd % 2 || V <= 0) return false;
-  // every weight stage must fit a ring slot
-  if ((size_t)I * 2 > kSlot || (size_t)H * 2 * 2 > kSlot) return false;
+  if (qkvd % 2 || V <= 0) return false;
+  // every K splits into column blocks of a multiple of 256 that fit a slot
+  for (int K : {H, qd, I})
+    if (phase_kblocks(K, 8) == 0 || phase_kblocks(K, 4) == 0) return false;
   const PGeo g = make_geo(kPMaxBatch, I > H ? I : H);
   return g.ring >= 2 && g.total <= kSmemMax;
 }
@@ -839,10 +1005,18 @@ static q2_status pdecode_launch(const PDecode& p, const CUtensorMap& kmap, const
     set_error("persistent decode: shared memory plan does not fit");
     return Q2_ERR_SHAPE;
   }
+  const int G = num_sms();
+  for (int N : {p.qkvd, p.H}) {  // rows per CTA with staged epilogue operands
+    const int R = phase_rows(N, G);
+    if ((N / R + G) / G * R > kEpiRows) {
+      set_error("persistent decode: too many rows per CTA for this device");
+      return Q2_ERR_SHAPE;
+    }
+  }
   Q2_CUDA_TRY(cudaFuncSetAttribute(pdecode_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    (int)g.total));
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(num_sms());
+  cfg.gridDim = dim3(G);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = g.total;
   cfg.stream = st;

@@ -67,6 +67,7 @@ struct PDecode {
   unsigned* sync;        // [pdecode_sync_words(L)] phase and merge counters, zero at launch
   unsigned long long* trace;  // optional [5L + 1][4] phase timestamps (see q2_model_time_kernels)
   int* err;              // bit 0: id outside the vocabulary; bit 1: a wait ran out
+  int l2_ahead;          // weight stages the producer pulls into L2 ahead of its ring
 };
 
 constexpr int kPConsumers = 8;
