@@ -20,7 +20,7 @@ import torch
 __all__ = [
     "Q2Error", "lib", "q2_version", "q2_check_device_error", "q2_add", "q2_argmax",
     "q2_argmax_noalloc", "q2_embedding",
-    "q2_linear", "q2_rms_norm", "q2_add_rms_norm", "q2_rope", "q2_self_attention", "q2_swiglu",
+    "q2_linear", "q2_test_tc_gemm", "q2_rms_norm", "q2_add_rms_norm", "q2_rope", "q2_self_attention", "q2_swiglu",
     "q2_rearrange", "Model", "W_KIND", "STATUS", "KCLASS",
 ]
 
@@ -60,6 +60,7 @@ _SIGS = {
     "q2_argmax_noalloc": [_VP, _VP, _VP, _SZ, _SZ, _I, _VP],
     "q2_embedding": [_VP, _VP, _VP, _SZ, _SZ, _SZ, _I, _VP],
     "q2_linear": [_VP, _VP, _VP, _VP, _SZ, _SZ, _SZ, _I, _VP],
+    "q2_test_tc_gemm": [_VP, _SZ, _I, _I, _VP, _VP, _VP, _SZ, _SZ, _SZ, _VP],
     "q2_rms_norm": [_VP, _VP, _VP, _SZ, _SZ, _F, _I, _VP],
     "q2_add_rms_norm": [_VP, _VP, _VP, _VP, _SZ, _SZ, _F, _I, _VP],
     "q2_rope": [_VP, _VP, _VP, _SZ, _SZ, _SZ, _F, _I, _VP],
@@ -190,6 +191,19 @@ def q2_linear(out, inp, weight, bias=None):
     N, K = weight.shape
     M = inp.numel() // K
     _call("q2_linear", _p(out), _p(inp), _p(weight), _p(bias), M, N, K, _dtype(inp), _stream())
+    return out
+
+
+TC_EPI = {"plain": 0, "swiglu": 1, "resid": 2}
+
+
+def q2_test_tc_gemm(out, x, weight, bias=None, epilogue="plain"):
+    """Test hook: the tcgen05 GEMM with one of its epilogues (see q2.h)."""
+    _dense(out, x, weight, bias)
+    N, K = weight.shape
+    M = x.numel() // K
+    _call("q2_test_tc_gemm", _p(out), out.shape[-1], _dtype(out), TC_EPI[epilogue], _p(x),
+          _p(weight), _p(bias), M, N, K, _stream())
     return out
 
 

@@ -7,6 +7,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "gemm_tc.h"
 
 namespace q2 {
 
@@ -121,6 +122,22 @@ q2_status q2_linear(void* out, const void* in, const void* weight, const void* b
   Q2_CHECK_ARG(K > 0, Q2_ERR_SHAPE, "linear: K must be positive");
   Q2_CHECK_ARG(M < (1u << 31) && N < (1u << 31) && K < (1u << 31), Q2_ERR_SHAPE, "linear: size too large");
   return launch_linear(out, in, weight, bias, (int)M, (int)N, (int)K, dtype, dtype, as_stream(stream), false);
+}
+
+q2_status q2_test_tc_gemm(void* out, size_t ldo, int out_dtype, int epilogue, const void* x,
+                          const void* w, const void* bias, size_t M, size_t N, size_t K,
+                          void* stream) {
+  clear_error();
+  Q2_CHECK_ARG(out_dtype == Q2_BF16 || out_dtype == Q2_F32, Q2_ERR_DTYPE, "tc gemm: bad out dtype");
+  Q2_CHECK_ARG(epilogue >= TC_EPI_PLAIN && epilogue <= TC_EPI_RESID, Q2_ERR_INVALID_ARG,
+               "tc gemm: bad epilogue");
+  Q2_CHECK_ARG(M == 0 || N == 0 || (out && x && w), Q2_ERR_INVALID_ARG, "tc gemm: NULL pointer");
+  Q2_CHECK_ARG(M < (1u << 31) && N < (1u << 31) && K < (1u << 31) && ldo < (1u << 31), Q2_ERR_SHAPE,
+               "tc gemm: size too large");
+  Q2_CHECK_ARG(K > 0 && K % 8 == 0, Q2_ERR_SHAPE, "tc gemm: K must be a positive multiple of 8");
+  cudaStream_t st = as_stream(stream);
+  Q2_TRY(tc_gemm(out, (int)ldo, out_dtype, epilogue, x, w, bias, (int)M, (int)N, (int)K, st));
+  return tc_check_error(st);
 }
 
 q2_status q2_rms_norm(void* out, const void* in, const void* weight, size_t M, size_t d, float eps,

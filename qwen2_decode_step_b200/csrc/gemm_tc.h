@@ -7,11 +7,23 @@
 
 namespace q2 {
 
-// Whether the tcgen05 path takes this linear (bf16 in, M large enough, K and
-// N multiples of the tile, pointers aligned for TMA).
+// Epilogues of tc_gemm (y = x w^T + bias, per output element):
+//   TC_EPI_PLAIN   out[m][n] = y (bf16 with one rounding, or fp32)
+//   TC_EPI_SWIGLU  w holds gate/up rows interleaved (row 2j gate j, row 2j + 1
+//                  up j): out[m][j] = silu(bf16(y[2j])) * bf16(y[2j + 1]), bf16
+//   TC_EPI_RESID   out[m][n] = bf16(out[m][n] + bf16(y)) (residual add in place)
+enum { TC_EPI_PLAIN = 0, TC_EPI_SWIGLU = 1, TC_EPI_RESID = 2 };
+
+// Whether the tcgen05 path takes this linear (bf16 operands, M >= 64 tokens,
+// N >= 128 features, K a multiple of 8, operands 16-byte aligned).
 bool tc_linear_supported(int M, int N, int K, const void* out, const void* in, const void* w);
 // out[M, N] (out_dtype) = in[M, K] . w[N, K]^T (+ bias[N]), bf16 operands.
 q2_status tc_linear(void* out, const void* in, const void* w, const void* bias, int M, int N, int K,
                     int out_dtype, cudaStream_t st, bool pdl);
+// The general form: output row stride `ldo` (elements) and an epilogue.
+q2_status tc_gemm(void* out, int ldo, int out_dtype, int epi, const void* x, const void* w,
+                  const void* bias, int M, int N, int K, cudaStream_t st);
+// Q2_ERR_CUDA (synchronising) if a pipeline wait in any tcgen05 GEMM ran out.
+q2_status tc_check_error(cudaStream_t st);
 
 }  // namespace q2
