@@ -304,10 +304,13 @@ q2_status tc_launch(const CUtensorMap& tw, const CUtensorMap& tx, const TcArgs& 
   return Q2_OK;
 }
 
+// One sticky device word per device for "a pipeline wait ran out" (a static
+// symbol: nothing is allocated, so launches may be captured in CUDA graphs).
+__device__ int g_tc_err;
+
 int* tc_err_flag() {
-  static int* flag = nullptr;  // one device word per process (errors are sticky)
-  if (!flag && cudaMalloc(&flag, sizeof(int)) == cudaSuccess) cudaMemset(flag, 0, sizeof(int));
-  return flag;
+  void* p = nullptr;
+  return cudaGetSymbolAddress(&p, g_tc_err) == cudaSuccess ? static_cast<int*>(p) : nullptr;
 }
 
 }  // namespace
@@ -361,6 +364,9 @@ q2_status tc_check_error(cudaStream_t st) {
   Q2_CUDA_TRY(cudaMemcpyAsync(&h, err, sizeof(int), cudaMemcpyDeviceToHost, st));
   Q2_CUDA_TRY(cudaStreamSynchronize(st));
   if (h) {
+    const int zero = 0;
+    cudaMemcpyAsync(err, &zero, sizeof(int), cudaMemcpyHostToDevice, st);
+    cudaStreamSynchronize(st);
     set_error("tcgen05 gemm: a pipeline wait ran out");
     return Q2_ERR_CUDA;
   }

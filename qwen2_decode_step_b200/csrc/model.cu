@@ -18,6 +18,7 @@
 #include "common.cuh"
 #include "decode.h"
 #include "kernels.h"
+#include "gemm_tc.h"
 #include "pdecode.h"
 #include <cstdlib>
 #include "tma.h"
@@ -222,10 +223,15 @@ int decode_splits(const q2_model* M, int rows) {
 
 // The decoder layers on x [T, H].  decode != 0: row t is the next token of
 // sequence t; else rows are positions pos0.. of sequence `seq`.  On return,
-// o holds the last layer's down-projection output (not yet added to x).
+// x holds the residual stream after the last layer.  bf16 with T >= 64 runs
+// the linears on the tcgen05 GEMM with fused epilogues (gate/up + SwiGLU,
+// o and down + the residual add in place); otherwise one kernel per operator.
 q2_status run_layers(q2_model* M, int T, int decode, int seq, int pos0, cudaStream_t st, bool pdl) {
   const q2_meta& m = M->m;
   const int H = m.hidden, I = m.intermediate, dt = M->dt;
+  const bool tc = dt == Q2_BF16 && tc_linear_supported(T, H, I, M->x, M->s, M->layers[0].wd) &&
+                  tc_linear_supported(T, H, M->qd, M->x, M->att, M->layers[0].wo) &&
+                  tc_linear_supported(T, 2 * I, H, M->s, M->h, M->layers[0].wgu);
   for (int l = 0; l < m.n_layers; ++l) {
     const LayerW& w = M->layers[l];
     if (l == 0)
@@ -267,14 +273,25 @@ q2_status run_layers(q2_model* M, int T, int decode, int seq, int pos0, cudaStre
     }
     TIMED(Q2_K_ATTN, launch_attention(a, nsplit, M->attn_scratch, dt, st, pdl));
 
-    TIMED(Q2_K_O, launch_linear(M->o, M->att, w.wo, nullptr, T, H, M->qd, dt, dt, st, pdl));
-    TIMED(Q2_K_NORM, launch_add_rms_norm(M->x, M->o, M->h, w.post_norm, T, H, m.eps, dt, st, pdl));
-    TIMED(Q2_K_GATE_UP, launch_linear(M->gu, M->h, w.wgu, nullptr, T, 2 * I, H, dt, dt, st, pdl));
-    TIMED(Q2_K_SWIGLU, launch_swiglu_interleaved(M->s, M->gu, T, I, dt, st, pdl));
-    TIMED(Q2_K_DOWN, launch_linear(M->o, M->s, w.wd, nullptr, T, H, I, dt, dt, st, pdl));
-    if (l + 1 < m.n_layers)
-      TIMED(Q2_K_NORM,
-            launch_add_rms_norm(M->x, M->o, M->h, M->layers[l + 1].in_norm, T, H, m.eps, dt, st, pdl));
+    if (tc) {
+      TIMED(Q2_K_O, tc_gemm(M->x, H, Q2_BF16, TC_EPI_RESID, M->att, w.wo, nullptr, T, H, M->qd, st));
+      TIMED(Q2_K_NORM, launch_add_rms_norm(M->x, nullptr, M->h, w.post_norm, T, H, m.eps, dt, st, pdl));
+      TIMED(Q2_K_GATE_UP, tc_gemm(M->s, I, Q2_BF16, TC_EPI_SWIGLU, M->h, w.wgu, nullptr, T, 2 * I, H, st));
+      TIMED(Q2_K_DOWN, tc_gemm(M->x, H, Q2_BF16, TC_EPI_RESID, M->s, w.wd, nullptr, T, H, I, st));
+      if (l + 1 < m.n_layers)
+        TIMED(Q2_K_NORM, launch_add_rms_norm(M->x, nullptr, M->h, M->layers[l + 1].in_norm, T, H, m.eps,
+                                             dt, st, pdl));
+    } else {
+      TIMED(Q2_K_O, launch_linear(M->o, M->att, w.wo, nullptr, T, H, M->qd, dt, dt, st, pdl));
+      TIMED(Q2_K_NORM, launch_add_rms_norm(M->x, M->o, M->h, w.post_norm, T, H, m.eps, dt, st, pdl));
+      TIMED(Q2_K_GATE_UP, launch_linear(M->gu, M->h, w.wgu, nullptr, T, 2 * I, H, dt, dt, st, pdl));
+      TIMED(Q2_K_SWIGLU, launch_swiglu_interleaved(M->s, M->gu, T, I, dt, st, pdl));
+      TIMED(Q2_K_DOWN, launch_linear(M->o, M->s, w.wd, nullptr, T, H, I, dt, dt, st, pdl));
+      // the residual add of the down projection (fused with the next RMSNorm)
+      TIMED(Q2_K_NORM, launch_add_rms_norm(M->x, M->o, l + 1 < m.n_layers ? M->h : nullptr,
+                                           l + 1 < m.n_layers ? M->layers[l + 1].in_norm : nullptr, T,
+                                           H, m.eps, dt, st, pdl));
+    }
   }
   return Q2_OK;
 }
@@ -489,7 +506,7 @@ q2_status decode_body(q2_model* M, int B, cudaStream_t st) {
   TIMED(Q2_K_EMBED,
         launch_embedding(M->x, M->d_ids, M->embed, B, m.vocab, m.hidden, M->dt, M->d_err, st, pdl));
   Q2_TRY(run_layers(M, B, 1, 0, 0, st, pdl));
-  Q2_TRY(run_head(M, 0, B, 0, st, pdl));
+  Q2_TRY(run_head(M, 0, B, 0, st, pdl, false));
   tbeg(M, Q2_K_OTHER, st);
   Q2_LAUNCH(inc_lens_kernel, dim3(1), dim3(64 * ((B + 63) / 64)), 0, st, pdl, M->d_len, B);
   tend(M, st);
@@ -903,7 +920,6 @@ q2_status q2_model_forward_hidden(q2_model* M, const void* x_in, int B, void* x_
     Q2_TRY(fused_layers(M, B, st));  // the residual stream ends in x
   } else {
     Q2_TRY(run_layers(M, B, 1, 0, 0, st, false));
-    Q2_TRY(launch_add_rms_norm(M->x, M->o, nullptr, nullptr, B, M->m.hidden, M->m.eps, M->dt, st, false));
   }
   Q2_CUDA_TRY(cudaMemcpyAsync(x_out, M->x, bytes, cudaMemcpyDeviceToDevice, st));
   Q2_LAUNCH(inc_lens_kernel, dim3(1), dim3(64 * ((B + 63) / 64)), 0, st, false, M->d_len, B);
@@ -938,7 +954,7 @@ q2_status q2_model_prefill(q2_model* M, const int64_t* ids, int batch, const int
       M->h_len[b] = pos0 + T;
       Q2_LAUNCH(set_len_kernel, dim3(1), dim3(1), 0, st, pdl, M->d_len, b, pos0 + T);
       if (c + T == n) {
-        Q2_TRY(run_head(M, T - 1, 1, b, st, pdl));
+        Q2_TRY(run_head(M, T - 1, 1, b, st, pdl, false));
         Q2_CUDA_TRY(cudaMemcpyAsync(next + b, M->d_next + b, sizeof(int64_t), cudaMemcpyDeviceToDevice, st));
         if (logits)
           Q2_CUDA_TRY(cudaMemcpyAsync(logits + (size_t)b * m.vocab, M->logits + (size_t)b * m.vocab,
@@ -1149,7 +1165,6 @@ q2_status q2_model_prefill_hidden(q2_model* M, int seq, const void* x_in, int T,
     const int pos0 = M->h_len[seq];
     Q2_CUDA_TRY(cudaMemcpyAsync(M->x, (const char*)x_in + c * row, Tc * row, cudaMemcpyDeviceToDevice, st));
     Q2_TRY(run_layers(M, Tc, 0, seq, pos0, st, true));
-    Q2_TRY(launch_add_rms_norm(M->x, M->o, nullptr, nullptr, Tc, M->m.hidden, M->m.eps, M->dt, st, true));
     Q2_CUDA_TRY(cudaMemcpyAsync((char*)x_out + c * row, M->x, Tc * row, cudaMemcpyDeviceToDevice, st));
     M->h_len[seq] = pos0 + Tc;
     Q2_LAUNCH(set_len_kernel, dim3(1), dim3(1), 0, st, true, M->d_len, seq, pos0 + Tc);
