@@ -124,11 +124,13 @@ q2_status q2_linear(void* out, const void* in, const void* weight, const void* b
  * fp32), 1 SwiGLU over interleaved gate/up rows (out[m, j] = silu(bf16(y[m,
  * 2j])) * bf16(y[m, 2j+1]), bf16), 2 residual add in place (out[m, n] =
  * bf16(out[m, n] + bf16(y[m, n])), bf16).  Requires M >= 1, K % 8 == 0 and
- * 16-byte aligned x and w; synchronises and returns Q2_ERR_CUDA if a pipeline
- * wait in the kernel ran out. */
+ * 16-byte aligned x and w.  allow_split != 0 lets a product with fewer tiles
+ * than SMs split K (through a temporary fp32 workspace the call allocates and
+ * frees).  Synchronises; returns Q2_ERR_CUDA if a pipeline wait in the kernel
+ * ran out. */
 q2_status q2_test_tc_gemm(void* out, size_t ldo, int out_dtype, int epilogue, const void* x,
                           const void* w, const void* bias, size_t M, size_t N, size_t K,
-                          void* stream);
+                          int allow_split, void* stream);
 
 /* rms_norm: out[m, :] = weight * in[m, :] / sqrt(mean(in[m, :]^2) + eps);
  * in, out [M, d]; weight [d].  out may alias in. */

@@ -60,7 +60,7 @@ _SIGS = {
     "q2_argmax_noalloc": [_VP, _VP, _VP, _SZ, _SZ, _I, _VP],
     "q2_embedding": [_VP, _VP, _VP, _SZ, _SZ, _SZ, _I, _VP],
     "q2_linear": [_VP, _VP, _VP, _VP, _SZ, _SZ, _SZ, _I, _VP],
-    "q2_test_tc_gemm": [_VP, _SZ, _I, _I, _VP, _VP, _VP, _SZ, _SZ, _SZ, _VP],
+    "q2_test_tc_gemm": [_VP, _SZ, _I, _I, _VP, _VP, _VP, _SZ, _SZ, _SZ, _I, _VP],
     "q2_rms_norm": [_VP, _VP, _VP, _SZ, _SZ, _F, _I, _VP],
     "q2_add_rms_norm": [_VP, _VP, _VP, _VP, _SZ, _SZ, _F, _I, _VP],
     "q2_rope": [_VP, _VP, _VP, _SZ, _SZ, _SZ, _F, _I, _VP],
@@ -197,13 +197,13 @@ def q2_linear(out, inp, weight, bias=None):
 TC_EPI = {"plain": 0, "swiglu": 1, "resid": 2}
 
 
-def q2_test_tc_gemm(out, x, weight, bias=None, epilogue="plain"):
+def q2_test_tc_gemm(out, x, weight, bias=None, epilogue="plain", split=False):
     """Test hook: the tcgen05 GEMM with one of its epilogues (see q2.h)."""
     _dense(out, x, weight, bias)
     N, K = weight.shape
     M = x.numel() // K
     _call("q2_test_tc_gemm", _p(out), out.shape[-1], _dtype(out), TC_EPI[epilogue], _p(x),
-          _p(weight), _p(bias), M, N, K, _stream())
+          _p(weight), _p(bias), M, N, K, 1 if split else 0, _stream())
     return out
 
 

@@ -126,7 +126,7 @@ q2_status q2_linear(void* out, const void* in, const void* weight, const void* b
 
 q2_status q2_test_tc_gemm(void* out, size_t ldo, int out_dtype, int epilogue, const void* x,
                           const void* w, const void* bias, size_t M, size_t N, size_t K,
-                          void* stream) {
+                          int allow_split, void* stream) {
   clear_error();
   Q2_CHECK_ARG(out_dtype == Q2_BF16 || out_dtype == Q2_F32, Q2_ERR_DTYPE, "tc gemm: bad out dtype");
   Q2_CHECK_ARG(epilogue >= TC_EPI_PLAIN && epilogue <= TC_EPI_RESID, Q2_ERR_INVALID_ARG,
@@ -136,8 +136,23 @@ q2_status q2_test_tc_gemm(void* out, size_t ldo, int out_dtype, int epilogue, co
                "tc gemm: size too large");
   Q2_CHECK_ARG(K > 0 && K % 8 == 0, Q2_ERR_SHAPE, "tc gemm: K must be a positive multiple of 8");
   cudaStream_t st = as_stream(stream);
-  Q2_TRY(tc_gemm(out, (int)ldo, out_dtype, epilogue, x, w, bias, (int)M, (int)N, (int)K, st));
-  return tc_check_error(st);
+  float* ws = nullptr;
+  size_t ws_bytes = 0;
+  if (allow_split && M && N) {
+    ws_bytes = (size_t)M * N * sizeof(float) * 16;
+    if (cudaMalloc(&ws, ws_bytes) != cudaSuccess) {
+      set_error("tc gemm: no memory for the split-K workspace");
+      return Q2_ERR_OOM;
+    }
+  }
+  q2_status s = tc_gemm(out, (int)ldo, out_dtype, epilogue, x, w, bias, (int)M, (int)N, (int)K, st,
+                        ws, ws_bytes);
+  if (s == Q2_OK) s = tc_check_error(st);
+  if (ws) {
+    cudaStreamSynchronize(st);
+    cudaFree(ws);
+  }
+  return s;
 }
 
 q2_status q2_rms_norm(void* out, const void* in, const void* weight, size_t M, size_t d, float eps,

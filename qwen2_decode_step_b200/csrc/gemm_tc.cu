@@ -117,6 +117,9 @@ struct TcArgs {
   int out_f32;       // 1: fp32 output, 0: bf16 (one rounding)
   int epi;           // TC_EPI_*
   int* err;          // bit 1: a wait ran out
+  int splits;        // K splits (1: the epilogue runs in this kernel)
+  int kb_per;        // k-blocks per split
+  float* ws;         // splits > 1: fp32 partial sums [splits][M][N]
 };
 
 template <int BN, int STAGES>
@@ -144,6 +147,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tiles_n = (a.N + kBM - 1) / kBM, tiles_m = (a.M + BN - 1) / BN;
   const int ntiles = tiles_n * tiles_m;
+  const int nitems = ntiles * a.splits;  // (tile, K split) work items
   const int kblocks = (a.K + kBK - 1) / kBK;
   constexpr uint32_t kCols = 2 * BN;  // two accumulators (a power of two >= 32)
 
@@ -175,9 +179,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (lane == 0) {
       int s = 0;
       uint32_t ph = 0;
-      for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
-        const int n0 = (t % tiles_n) * kBM, m0 = (t / tiles_n) * BN;
-        for (int kb = 0; kb < kblocks; ++kb) {
+      for (int t = blockIdx.x; t < nitems; t += gridDim.x) {
+        const int tile = t % ntiles, kb0 = (t / ntiles) * a.kb_per;
+        const int kb1 = min(kblocks, kb0 + a.kb_per);
+        const int n0 = (tile % tiles_n) * kBM, m0 = (tile / tiles_n) * BN;
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!tc_wait(&empty[s], ph ^ 1u)) atomicOr(a.err, 2);
           uint8_t* st = smem + s * SM::kStage;
           mbar_arrive_expect_tx(&full[s], (uint32_t)SM::kStage);
@@ -197,20 +203,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       int s = 0;
       uint32_t ph = 0;
       int it = 0;
-      for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
+      for (int t = blockIdx.x; t < nitems; t += gridDim.x, ++it) {
         const int acc = it & 1;
+        const int kb0 = (t / ntiles) * a.kb_per, kb1 = min(kblocks, kb0 + a.kb_per);
         // the epilogue has drained this accumulator (fresh barriers pass at once)
         if (!tc_wait(&acc_empty[acc], (uint32_t)(((it >> 1) & 1) ^ 1))) atomicOr(a.err, 2);
         tc_fence_after();
         const uint32_t d = tmem + (uint32_t)(acc * BN);
-        for (int kb = 0; kb < kblocks; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!tc_wait(&full[s], ph)) atomicOr(a.err, 2);
           tc_fence_after();
           const uint8_t* st = smem + s * SM::kStage;
           const uint64_t da = sw128_desc(st), db = sw128_desc(st + SM::kA);
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k)  // 16 bf16 = 32 bytes along the swizzle atom
-            tc_mma(d, da + (uint64_t)(2 * k), db + (uint64_t)(2 * k), idesc, (kb | k) != 0);
+            tc_mma(d, da + (uint64_t)(2 * k), db + (uint64_t)(2 * k), idesc, kb != kb0 || k != 0);
           tc_commit(&empty[s]);  // the stage is free once these MMAs are done
           if (++s == STAGES) {
             s = 0;
@@ -224,9 +231,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // the TMEM lane quarter this warp may access
     int it = 0;
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
+    for (int t = blockIdx.x; t < nitems; t += gridDim.x, ++it) {
       const int acc = it & 1;
-      const int n0 = (t % tiles_n) * kBM, m0 = (t / tiles_n) * BN;
+      const int tile = t % ntiles, split = t / ntiles;
+      const int n0 = (tile % tiles_n) * kBM, m0 = (tile / tiles_n) * BN;
       if (lane == 0 && !tc_wait(&acc_full[acc], (uint32_t)((it >> 1) & 1))) atomicOr(a.err, 2);
       __syncwarp();
       tc_fence_after();
@@ -237,7 +245,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int c = 0; c < BN; c += 32) {
         float v[32];
         tmem_ld32(tbase + (uint32_t)c, v);
-        if (a.epi == TC_EPI_SWIGLU) {
+        if (a.splits > 1) {  // partial sums; the finishing kernel adds them in split order
+          float* w = a.ws + (size_t)split * a.M * a.N;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int m = m0 + c + j;
+            if (m < a.M && n < a.N) w[(size_t)m * a.N + n] = v[j];
+          }
+        } else if (a.epi == TC_EPI_SWIGLU) {
           // rows 2j (gate) and 2j + 1 (up) sit in adjacent lanes
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
@@ -288,14 +303,58 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
 }
 
+// Split-K finish: y = sum of the splits' partials in split order (+ bias),
+// then the epilogue.  One thread per output element (per gate/up pair for
+// SwiGLU).
+__global__ void tc_finish_kernel(const TcArgs a) {
+  const int N = a.N;
+  const int cols = a.epi == TC_EPI_SWIGLU ? N / 2 : N;
+  const size_t total = (size_t)a.M * cols;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const int m = (int)(i / cols), c = (int)(i % cols);
+    if (a.epi == TC_EPI_SWIGLU) {
+      float g = 0.f, u = 0.f;
+      for (int s = 0; s < a.splits; ++s) {
+        const float* w = a.ws + ((size_t)s * a.M + m) * N;
+        g += w[2 * c];
+        u += w[2 * c + 1];
+      }
+      if (a.bias) {
+        g += __bfloat162float(a.bias[2 * c]);
+        u += __bfloat162float(a.bias[2 * c + 1]);
+      }
+      const float gv = round_st<bf16>(g), uv = round_st<bf16>(u);
+      reinterpret_cast<bf16*>(a.out)[(size_t)m * a.ldo + c] = from_f<bf16>(uv * (gv / (1.0f + expf(-gv))));
+    } else {
+      float y = 0.f;
+      for (int s = 0; s < a.splits; ++s) y += a.ws[((size_t)s * a.M + m) * N + c];
+      if (a.bias) y += __bfloat162float(a.bias[c]);
+      if (a.epi == TC_EPI_RESID) {
+        bf16* o = reinterpret_cast<bf16*>(a.out) + (size_t)m * a.ldo + c;
+        *o = from_f<bf16>(__bfloat162float(*o) + round_st<bf16>(y));
+      } else if (a.out_f32) {
+        reinterpret_cast<float*>(a.out)[(size_t)m * a.ldo + c] = y;
+      } else {
+        reinterpret_cast<bf16*>(a.out)[(size_t)m * a.ldo + c] = from_f<bf16>(y);
+      }
+    }
+  }
+}
+
 template <int BN, int STAGES>
 q2_status tc_launch(const CUtensorMap& tw, const CUtensorMap& tx, const TcArgs& a, cudaStream_t st) {
   using SM = TcSmem<BN, STAGES>;
   Q2_CUDA_TRY(cudaFuncSetAttribute(tc_gemm_kernel<BN, STAGES>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SM::kTotal));
-  const int tiles = ((a.N + kBM - 1) / kBM) * ((a.M + BN - 1) / BN);
-  const int grid = tiles < num_sms() ? tiles : num_sms();
+  const int items = ((a.N + kBM - 1) / kBM) * ((a.M + BN - 1) / BN) * a.splits;
+  const int grid = items < num_sms() ? items : num_sms();
   tc_gemm_kernel<BN, STAGES><<<grid, kTcThreads, SM::kTotal, st>>>(tw, tx, a);
+  if (a.splits > 1) {
+    const size_t total = (size_t)a.M * (a.epi == TC_EPI_SWIGLU ? a.N / 2 : a.N);
+    const int blocks = (int)((total + 255) / 256 < (size_t)num_sms() * 8 ? (total + 255) / 256 : num_sms() * 8);
+    tc_finish_kernel<<<blocks, 256, 0, st>>>(a);
+  }
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_error(std::string("tcgen05 gemm launch: ") + cudaGetErrorString(e));
@@ -323,7 +382,7 @@ bool tc_linear_supported(int M, int N, int K, const void* out, const void* in, c
 }
 
 q2_status tc_gemm(void* out, int ldo, int out_dtype, int epi, const void* x, const void* w,
-                  const void* bias, int M, int N, int K, cudaStream_t st) {
+                  const void* bias, int M, int N, int K, cudaStream_t st, float* ws, size_t ws_bytes) {
   if (M <= 0 || N <= 0) return Q2_OK;
   if (K % 8 != 0 || (reinterpret_cast<uintptr_t>(x) & 15) || (reinterpret_cast<uintptr_t>(w) & 15)) {
     set_error("tcgen05 gemm: K must be a multiple of 8 and operands 16-byte aligned");
@@ -349,6 +408,21 @@ q2_status tc_gemm(void* out, int ldo, int out_dtype, int epi, const void* x, con
   a.epi = epi;
   a.err = err;
   const int bn = M >= 256 ? 256 : (M >= 128 ? 128 : 64);
+  // Split K when the tiles alone would leave SMs idle (few output features,
+  // few tokens): aim for one work item per SM, at least two k-blocks each,
+  // within the workspace.
+  const int tiles = ((N + kBM - 1) / kBM) * ((M + bn - 1) / bn);
+  const int kblocks = (K + kBK - 1) / kBK;
+  int splits = 1;
+  if (ws != nullptr && tiles < num_sms()) {
+    splits = (num_sms() + tiles - 1) / tiles;
+    if (splits > kblocks / 2) splits = kblocks / 2;
+    while (splits > 1 && (size_t)splits * M * N * sizeof(float) > ws_bytes) --splits;
+    if (splits < 1) splits = 1;
+  }
+  a.kb_per = (kblocks + splits - 1) / splits;
+  a.splits = (kblocks + a.kb_per - 1) / a.kb_per;  // every split has a k-block
+  a.ws = ws;
   CUtensorMap tw, tx;
   Q2_TRY(make_tmap_2d_bf16(&tw, w, (uint64_t)N, (uint64_t)K, (uint64_t)K * 2, kBM, kBK, 128));
   Q2_TRY(make_tmap_2d_bf16(&tx, x, (uint64_t)M, (uint64_t)K, (uint64_t)K * 2, (uint32_t)bn, kBK, 128));
@@ -376,7 +450,7 @@ q2_status tc_check_error(cudaStream_t st) {
 q2_status tc_linear(void* out, const void* in, const void* w, const void* bias, int M, int N, int K,
                     int out_dtype, cudaStream_t st, bool pdl) {
   (void)pdl;
-  return tc_gemm(out, N, out_dtype, TC_EPI_PLAIN, in, w, bias, M, N, K, st);
+  return tc_gemm(out, N, out_dtype, TC_EPI_PLAIN, in, w, bias, M, N, K, st, nullptr, 0);
 }
 
 }  // namespace q2

@@ -92,6 +92,8 @@ struct q2_model {
   PLayer* d_layers = nullptr;      // device copy of the per-layer weight pointers
   unsigned* d_sync = nullptr;      // persistent step phase counters
   unsigned long long* d_trace = nullptr;  // persistent step phase timestamps [5L + 1][4]
+  float* tc_ws = nullptr;                 // split-K partial sums of the tcgen05 GEMM
+  size_t tc_ws_bytes = 0;
   CUtensorMap kmap{}, vmap{};      // the K and V caches as 2-D [rows, hd] tensors
 
   cudaStream_t cap = nullptr;
@@ -236,7 +238,11 @@ q2_status run_layers(q2_model* M, int T, int decode, int seq, int pos0, cudaStre
     const LayerW& w = M->layers[l];
     if (l == 0)
       TIMED(Q2_K_NORM, launch_add_rms_norm(M->x, nullptr, M->h, w.in_norm, T, H, m.eps, dt, st, pdl));
-    TIMED(Q2_K_QKV, launch_linear(M->qkv, M->h, w.wqkv, w.bqkv, T, M->qkvd, H, dt, dt, st, pdl));
+    if (tc)
+      TIMED(Q2_K_QKV, tc_gemm(M->qkv, M->qkvd, Q2_BF16, TC_EPI_PLAIN, M->h, w.wqkv, w.bqkv, T, M->qkvd, H,
+                              st, M->tc_ws, M->tc_ws_bytes));
+    else
+      TIMED(Q2_K_QKV, launch_linear(M->qkv, M->h, w.wqkv, w.bqkv, T, M->qkvd, H, dt, dt, st, pdl));
     TIMED(Q2_K_ROPE_KV, launch_rope_kv(M, l, T, M->d_len, decode, seq, pos0, st, pdl));
 
     AttnRows a = {};
@@ -274,10 +280,13 @@ q2_status run_layers(q2_model* M, int T, int decode, int seq, int pos0, cudaStre
     TIMED(Q2_K_ATTN, launch_attention(a, nsplit, M->attn_scratch, dt, st, pdl));
 
     if (tc) {
-      TIMED(Q2_K_O, tc_gemm(M->x, H, Q2_BF16, TC_EPI_RESID, M->att, w.wo, nullptr, T, H, M->qd, st));
+      TIMED(Q2_K_O, tc_gemm(M->x, H, Q2_BF16, TC_EPI_RESID, M->att, w.wo, nullptr, T, H, M->qd, st, M->tc_ws,
+                              M->tc_ws_bytes));
       TIMED(Q2_K_NORM, launch_add_rms_norm(M->x, nullptr, M->h, w.post_norm, T, H, m.eps, dt, st, pdl));
-      TIMED(Q2_K_GATE_UP, tc_gemm(M->s, I, Q2_BF16, TC_EPI_SWIGLU, M->h, w.wgu, nullptr, T, 2 * I, H, st));
-      TIMED(Q2_K_DOWN, tc_gemm(M->x, H, Q2_BF16, TC_EPI_RESID, M->s, w.wd, nullptr, T, H, I, st));
+      TIMED(Q2_K_GATE_UP, tc_gemm(M->s, I, Q2_BF16, TC_EPI_SWIGLU, M->h, w.wgu, nullptr, T, 2 * I, H, st,
+                                    M->tc_ws, M->tc_ws_bytes));
+      TIMED(Q2_K_DOWN, tc_gemm(M->x, H, Q2_BF16, TC_EPI_RESID, M->s, w.wd, nullptr, T, H, I, st, M->tc_ws,
+                                 M->tc_ws_bytes));
       if (l + 1 < m.n_layers)
         TIMED(Q2_K_NORM, launch_add_rms_norm(M->x, nullptr, M->h, M->layers[l + 1].in_norm, T, H, m.eps,
                                              dt, st, pdl));
@@ -696,6 +705,13 @@ q2_status q2_model_create(const q2_meta* meta, int device, q2_model** out) {
   al.push_back({(void**)&M->d_sync, pdecode_sync_words(m.n_layers) * sizeof(unsigned)});
   al.push_back({(void**)&M->d_layers, (size_t)m.n_layers * sizeof(PLayer)});
   al.push_back({(void**)&M->d_trace, (5 * (size_t)m.n_layers + 1) * 4 * sizeof(unsigned long long)});
+  if (M->dt == Q2_BF16) {
+    // Split-K partial sums of the tcgen05 GEMM: a product is split only while
+    // it has fewer tiles than SMs, so splits x tokens x features stays near
+    // SMs x 256 x 128 x 4 bytes (~20 MB); calls that need more split less.
+    M->tc_ws_bytes = (size_t)40 << 20;
+    al.push_back({(void**)&M->tc_ws, M->tc_ws_bytes});
+  }
   size_t abytes = 0;
   for (auto& p : al) abytes += align_up(p.second ? p.second : 1, 256);
   if (cudaMalloc(&M->abuf, abytes) != cudaSuccess) {

@@ -35,13 +35,27 @@ def cuda(t):
     (512, 1536, 8960),    # the down projection, long K
 ])
 @pytest.mark.parametrize("bias", [False, True])
-def test_tc_gemm_plain_bf16(M, N, K, bias):
+@pytest.mark.parametrize("split", [False, True])
+def test_tc_gemm_plain_bf16(M, N, K, bias, split):
     x = normal((M, K), 1.0, 101, "bf16")
     w = normal((N, K), 0.02, 102, "bf16")
     b = normal((N,), 0.01, 103, "bf16") if bias else None
     out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
-    q2.q2_test_tc_gemm(out, cuda(x), cuda(w), cuda(b))
-    assert_op_close(out, oracle.linear(x, w, b), f"tc gemm {M}x{N}x{K}")
+    q2.q2_test_tc_gemm(out, cuda(x), cuda(w), cuda(b), split=split)
+    assert_op_close(out, oracle.linear(x, w, b), f"tc gemm {M}x{N}x{K} split={split}")
+
+
+def test_tc_gemm_split_k_is_deterministic():
+    """Split-K partials are added in split order: repeated calls agree bit for bit."""
+    M, N, K = 64, 1536, 8960
+    x = cuda(normal((M, K), 1.0, 161, "bf16"))
+    w = cuda(normal((N, K), 0.02, 162, "bf16"))
+    outs = []
+    for _ in range(3):
+        out = torch.empty((M, N), dtype=torch.float32, device="cuda")
+        q2.q2_test_tc_gemm(out, x, w, split=True)
+        outs.append(out)
+    assert bits_equal(outs[0], outs[1]) and bits_equal(outs[0], outs[2])
 
 
 @pytest.mark.parametrize("M,N,K", [(64, 256, 1536), (257, 640, 1536)])
@@ -77,7 +91,7 @@ def test_tc_gemm_swiglu_epilogue(M):
     wu = normal((I, K), 0.02, 133, "bf16")
     w = torch.stack([wg, wu], dim=1).reshape(2 * I, K)  # row 2j gate j, 2j + 1 up j
     out = torch.empty((M, I), dtype=torch.bfloat16, device="cuda")
-    q2.q2_test_tc_gemm(out, cuda(x), cuda(w), epilogue="swiglu")
+    q2.q2_test_tc_gemm(out, cuda(x), cuda(w), epilogue="swiglu", split=M == 64)
     ref = oracle.swiglu(oracle.linear(x, wg), oracle.linear(x, wu))
     # Two operators in one kernel: the gate and up values are each rounded to
     # bf16 from an fp32 (not fp64) sum, so either may land one bf16 ulp away
@@ -93,7 +107,7 @@ def test_tc_gemm_residual_epilogue(M):
     w = normal((N, K), 0.02, 142, "bf16")
     r = normal((M, N), 1.0, 143, "bf16")
     out = cuda(r.clone())
-    q2.q2_test_tc_gemm(out, cuda(x), cuda(w), epilogue="resid")
+    q2.q2_test_tc_gemm(out, cuda(x), cuda(w), epilogue="resid", split=M == 64)
     ref = oracle.add(r, oracle.linear(x, w))
     # Two operators in one kernel (linear rounded to bf16, then the add): the
     # linear's rounding may differ by one ulp from the oracle's, so the
