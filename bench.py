@@ -156,10 +156,17 @@ def decode_step_bytes(s, batch: int, ctx: float) -> float:
     return w + batch * (ctx + 1) * kv_per_pos + batch * s.hidden * es
 
 
-def kernel_src_hash() -> str:
+# The source files each profiled kernel is built from: a recorded DRAM
+# traffic figure stands only while these are unchanged.
+KERNEL_SOURCES = {
+    "gate_up": ["decode.cu", "decode.h", "common.cuh", "tma.h", "kernels.h"],
+}
+
+
+def kernel_src_hash(kernel: str = "gate_up") -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "qwen2_decode_step_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
+    for fn in KERNEL_SOURCES[kernel]:
         h.update(open(os.path.join(csrc, fn), "rb").read())
     return h.hexdigest()[:16]
 
@@ -172,7 +179,7 @@ def recorded_traffic(kernel: str, workload: str):
         return None
     d = json.load(open(p))
     e = d.get(f"{kernel}@{workload}")
-    if not e or e.get("src_hash") != kernel_src_hash():
+    if not e or e.get("src_hash") != kernel_src_hash(kernel):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -354,6 +361,9 @@ def run_ours(args, dist: Dist):
 
     pk, pk_kind = peaks()
     hbm = float(pk["hbm_gbs"])
+    gemms = None
+    if not args.no_prefill_gemms:
+        gemms = prefill_gemm_rates(shape, args.prefill_gemm_tokens, float(pk["bf16_tflops"]))
     gu_ms, gu_n = ktimes["gate_up"]
     gu_bytes = 2 * shape.intermediate * shape.hidden * 2 + shape.hidden * 2 + 2 * shape.intermediate * 2
     achieved = gu_bytes / (gu_ms / 1e3) / 1e9 if gu_ms > 0 else None
@@ -385,6 +395,9 @@ def run_ours(args, dist: Dist):
         "gpu_launches": kernels_per_step * args.steps,
         "kernels_per_step": kernels_per_step,
         "prefill": {"tokens": prompt_len, "ms": pre_ms, "tok_s": prompt_len / (pre_ms / 1e3)},
+        "prefill_gemms": gemms and {"tokens_per_chunk": args.prefill_gemm_tokens,
+                                    "peak_tflops": float(pk["bf16_tflops"]), "peak_kind": pk_kind,
+                                    "kernel": "tc_gemm_kernel (tcgen05, TMEM)", "shapes": gemms},
         "e2e": {"value": 1 * dist.world / (e2e_ms / 1e3), "unit": "tok/s", "h2d_bytes_per_step": 8,
                 "d2h_bytes_per_step": 8, "ms_per_step": e2e_ms,
                 "api": "q2_model_decode_step_host (pinned host ids -> host next)"},
@@ -399,6 +412,29 @@ def run_ours(args, dist: Dist):
     if dist.rank == 0:
         print(json.dumps(line), flush=True)
     dist.close()
+
+
+def prefill_gemm_rates(shape, tokens: int, peak_tflops: float, reps: int = 10):
+    """The tcgen05 GEMM on the prefill linears of one `tokens`-token chunk
+    (synthetic bf16 operands resident on the device), timed with CUDA events
+    on the current stream: TFLOP/s and the fraction of the measured bf16 peak."""
+    import qwen2_decode_step_b200 as q2
+    H, I, qkvd = shape.hidden, shape.intermediate, shape.q_dim + 2 * shape.kv_dim
+    g = torch.Generator(device="cuda")
+    g.manual_seed(4242)
+    out = {}
+    for name, N, K in (("qkv", qkvd, H), ("o", H, shape.q_dim), ("gate_up", 2 * I, H), ("down", H, I)):
+        x = torch.randn(tokens, K, device="cuda", generator=g).bfloat16()
+        w = (torch.randn(N, K, device="cuda", generator=g) * 0.02).bfloat16()
+        y = torch.empty(tokens, N, device="cuda", dtype=torch.bfloat16)
+        for _ in range(3):
+            q2.q2_linear(y, x, w)
+        ms = cuda_time(lambda: q2.q2_linear(y, x, w), reps) / reps
+        tf = 2.0 * tokens * N * K / (ms / 1e3) / 1e12
+        out[name] = {"M": tokens, "N": N, "K": K, "ms": ms, "tflops": tf, "frac": tf / peak_tflops}
+        del x, w, y
+    q2.q2_check_device_error()
+    return out
 
 
 def cuda_time_b64(model, bufs, n):
@@ -421,6 +457,9 @@ def main():
     ap.add_argument("--b64-steps", type=int, default=32)
     ap.add_argument("--no-b64", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill-gemms", action="store_true")
+    ap.add_argument("--prefill-gemm-tokens", type=int, default=4096,
+                    help="tokens of the prefill chunk whose linears are timed (the model's chunk size)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     args = ap.parse_args()
     if args.warmup < 3:
