@@ -70,5 +70,10 @@ struct DAttn {
 bool dattn_supported(int nh, int nkv, int hd);
 q2_status launch_dattn(const DAttn& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
                        cudaStream_t st);
+// The same attention with the dot products on the tensor cores (mma.sync):
+// head dim 128, up to 8 query heads per kv head, any batch, nsplit <= 64.
+bool dattn_mma_supported(int nh, int nkv, int hd, int nsplit);
+q2_status launch_dattn_mma(const DAttn& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
+                           cudaStream_t st);
 
 }  // namespace q2

@@ -262,6 +262,30 @@ q2_status run_layers(q2_model* M, int T, int decode, int seq, int pos0, cudaStre
     a.hd = m.head_dim;
     a.scale = 1.0f / sqrtf((float)m.head_dim);
     int nsplit;
+    if (decode && M->fused && dt == Q2_BF16 &&
+        dattn_mma_supported(m.n_heads, m.n_kv_heads, m.head_dim, decode_splits(M, T))) {
+      // decode rows over the cache: the tensor-core attention
+      DAttn d = {};
+      d.q = M->qb;
+      d.q_stride = M->qd;
+      d.out = M->att;
+      d.nsplit = decode_splits(M, T);
+      d.part_o = (float*)M->attn_scratch;
+      d.part_ml = d.part_o + (size_t)T * m.n_heads * d.nsplit * m.head_dim;
+      d.counters = M->d_counters;
+      d.lens = M->d_len;
+      d.B = T;
+      d.nh = m.n_heads;
+      d.nkv = m.n_kv_heads;
+      d.hd = m.head_dim;
+      d.max_seq = m.max_seq;
+      d.Bmax = m.max_batch;
+      d.layer = l;
+      d.scale = 1.0f / sqrtf((float)m.head_dim);
+      d.err = M->d_err;
+      TIMED(Q2_K_ATTN, launch_dattn_mma(d, M->kmap, M->vmap, st));
+      goto attention_done;
+    }
     if (decode) {
       a.base = 1;
       a.row_step = 0;
@@ -278,6 +302,7 @@ q2_status run_layers(q2_model* M, int T, int decode, int seq, int pos0, cudaStre
       nsplit = attn_splits(T, m.n_kv_heads, pos0 + T);
     }
     TIMED(Q2_K_ATTN, launch_attention(a, nsplit, M->attn_scratch, dt, st, pdl));
+  attention_done:
 
     if (tc) {
       TIMED(Q2_K_O, tc_gemm(M->x, H, Q2_BF16, TC_EPI_RESID, M->att, w.wo, nullptr, T, H, M->qd, st, M->tc_ws,
@@ -438,7 +463,10 @@ q2_status fused_layers(q2_model* M, int B, cudaStream_t st) {
     a.layer = l;
     a.scale = 1.0f / sqrtf((float)m.head_dim);
     a.err = M->d_err;
-    TIMED(Q2_K_ATTN, launch_dattn(a, M->kmap, M->vmap, st));
+    if (dattn_mma_supported(a.nh, a.nkv, a.hd, a.nsplit))
+      TIMED(Q2_K_ATTN, launch_dattn_mma(a, M->kmap, M->vmap, st));
+    else
+      TIMED(Q2_K_ATTN, launch_dattn(a, M->kmap, M->vmap, st));
 
     DGemv o = {};
     o.w = w.wo;
