@@ -270,6 +270,7 @@ static q2_status attn_t(const AttnRows& a, int nsplit, void* scratch, cudaStream
 
 q2_status launch_attention(const AttnRows& a, int nsplit, void* scratch, int dtype,
                            cudaStream_t st, bool pdl) {
+  if (attn_prefill_mma_supported(a, dtype)) return launch_attn_prefill_mma(a, st, pdl);
   if (a.rows == 0) return Q2_OK;
   if (a.nkv <= 0 || a.nh % a.nkv != 0 || a.nh / a.nkv > kGMax) {
     set_error("attention: need nh % nkv == 0 and nh / nkv <= 8");

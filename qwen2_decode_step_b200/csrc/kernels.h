@@ -69,5 +69,9 @@ int attn_splits(int rows, int nkv, int max_keys);
 size_t attn_scratch_bytes(int rows, int nh, int hd, int nsplit);
 q2_status launch_attention(const AttnRows& a, int nsplit, void* scratch, int dtype,
                            cudaStream_t st, bool pdl);
+// Rows of one sequence (prefill), bf16, head dim 128: flash-attention on the
+// tensor cores (launch_attention takes it by itself when it applies).
+bool attn_prefill_mma_supported(const AttnRows& a, int dtype);
+q2_status launch_attn_prefill_mma(const AttnRows& a, cudaStream_t st, bool pdl);
 
 }  // namespace q2

@@ -157,14 +157,19 @@ def _attn_case(dt, S, T, nh, nkv, hd, seed):
     (16, 16, 4, 2, 32),        # tiny-model shape
     (5, 300, 8, 8, 64),        # plain MHA
     (3, 77, 8, 1, 64),         # MQA (group 8)
+    (16, 16, 12, 2, 128),      # one warp's rows (bf16: tensor-core prefill kernel)
+    (128, 128, 12, 2, 128),    # two full row blocks, square causal
+    (100, 612, 12, 2, 128),    # prefill chunk after 512 cached positions, ragged
+    (300, 4096, 12, 2, 128),   # long cache, ragged row block and key tile
 ])
 def test_self_attention(dt, S, T, nh, nkv, hd):
     out, ref = _attn_case(dt, S, T, nh, nkv, hd, 20)
     assert_op_close(out, ref, f"attention S={S} T={T}")
 
 
-def test_self_attention_constant_v_and_future_independence():
-    S, T, nh, nkv, hd = 4, 300, 12, 2, 128
+@pytest.mark.parametrize("S", [4, 40])  # 40 rows: the tensor-core prefill kernel
+def test_self_attention_constant_v_and_future_independence(S):
+    T, nh, nkv, hd = 300, 12, 2, 128
     q = normal((S, nh, hd), 2.0, 30, "bf16")
     k = normal((T, nkv, hd), 2.0, 31, "bf16")
     v = torch.ones((T, nkv, hd), dtype=torch.bfloat16)
