@@ -9,14 +9,15 @@
 // thread of the epilogue owns one output feature and writes, token by token,
 // 32 consecutive features per warp store.
 //
-// Warp roles (192 threads, one CTA per SM, persistent over the tiles):
+// Warp roles (320 threads, one CTA per SM, persistent over the tiles):
 //   warp 0      TMA producer: a 128 x 64 weight box and a BN x 64 token box
 //               per k-block into a kStages ring (full/empty mbarriers)
 //   warp 1      allocates tensor memory and issues the MMAs (one thread);
 //               tcgen05.commit frees a ring stage and, after a tile's last
 //               k-block, publishes the accumulator
-//   warps 2-5   epilogue: tcgen05.ld of the warp's 32 TMEM lanes, bias,
-//               conversion, stores; then release the accumulator
+//   warps 2-9   epilogue: two warps per 32-lane TMEM quarter, each taking
+//               alternate 32-column chunks: tcgen05.ld, bias, the epilogue
+//               operator, conversion, stores; then release the accumulator
 // The accumulator is double-buffered in tensor memory (2 x BN fp32 columns),
 // so the epilogue of one tile overlaps the MMAs of the next.  Every wait is
 // bounded: a wait that runs out records an error flag and the kernel carries
@@ -33,7 +34,8 @@ namespace {
 
 constexpr int kBM = 128;       // output features per tile (MMA M)
 constexpr int kBK = 64;        // k per stage: one 128-byte swizzle atom of bf16
-constexpr int kTcThreads = 192;
+constexpr int kTcEpiWarps = 8;                     // two per TMEM lane quarter
+constexpr int kTcThreads = (2 + kTcEpiWarps) * 32;  // + the producer and MMA warps
 constexpr uint64_t kTcDeadlineNs = 2000ull * 1000 * 1000;  // 2 s
 
 __device__ __forceinline__ uint64_t tc_gtimer() {
@@ -158,7 +160,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], 4);  // one arrival per epilogue warp
+      mbar_init(&acc_empty[i], kTcEpiWarps);  // one arrival per epilogue warp
     }
     fence_mbar_init();
   }
@@ -229,7 +231,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // the TMEM lane quarter this warp may access
+    const int q = warp & 3;                    // the TMEM lane quarter this warp may access
+    const int half = (warp - 2) / 4;           // which alternate 32-column chunks it takes
     int it = 0;
     for (int t = blockIdx.x; t < nitems; t += gridDim.x, ++it) {
       const int acc = it & 1;
@@ -242,7 +245,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const float bn = (a.bias != nullptr && n < a.N) ? __bfloat162float(a.bias[n]) : 0.f;
       const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(acc * BN);
 #pragma unroll 1
-      for (int c = 0; c < BN; c += 32) {
+      for (int c = 32 * half; c < BN; c += 64) {
         float v[32];
         tmem_ld32(tbase + (uint32_t)c, v);
         if (a.splits > 1) {  // partial sums; the finishing kernel adds them in split order
@@ -253,26 +256,32 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (m < a.M && n < a.N) w[(size_t)m * a.N + n] = v[j];
           }
         } else if (a.epi == TC_EPI_SWIGLU) {
-          // rows 2j (gate) and 2j + 1 (up) sit in adjacent lanes
+          // Rows 2i (gate) and 2i + 1 (up) sit in adjacent lanes.  For each
+          // pair of tokens the even lane finishes the first and the odd lane
+          // the second, after swapping the one value each is missing.
+          const bool odd = (lane & 1) != 0;
+          const bool pair_ok = (n | 1) < a.N;
+          bf16* col = reinterpret_cast<bf16*>(a.out) + (n >> 1);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float gv = round_st<bf16>(v[j] + bn);
-            const float uv = __shfl_down_sync(0xffffffffu, gv, 1);
-            const int m = m0 + c + j;
-            if ((lane & 1) == 0 && m < a.M && n + 1 < a.N) {
-              const float sg = uv * (gv / (1.0f + expf(-gv)));
-              reinterpret_cast<bf16*>(a.out)[(size_t)m * a.ldo + (n >> 1)] = from_f<bf16>(sg);
-            }
+          for (int j = 0; j < 32; j += 2) {
+            const float mine0 = round_st<bf16>(v[j] + bn), mine1 = round_st<bf16>(v[j + 1] + bn);
+            const float got = __shfl_xor_sync(0xffffffffu, odd ? mine0 : mine1, 1);
+            const float gv = odd ? got : mine0, uv = odd ? mine1 : got;
+            const int m = m0 + c + j + (odd ? 1 : 0);
+            if (pair_ok && m < a.M)
+              col[(size_t)m * a.ldo] = from_f<bf16>(uv * (gv / (1.0f + expf(-gv))));
           }
         } else if (a.epi == TC_EPI_RESID) {
+          // all 32 residual loads first (they do not depend on the stores)
+          bf16* col = reinterpret_cast<bf16*>(a.out) + (size_t)(m0 + c) * a.ldo + n;
+          const bool nok = n < a.N;
+          float xr[32];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int m = m0 + c + j;
-            if (m < a.M && n < a.N) {
-              bf16* o = reinterpret_cast<bf16*>(a.out) + (size_t)m * a.ldo + n;
-              *o = from_f<bf16>(__bfloat162float(*o) + round_st<bf16>(v[j] + bn));
-            }
-          }
+          for (int j = 0; j < 32; ++j)
+            xr[j] = (nok && m0 + c + j < a.M) ? __bfloat162float(col[(size_t)j * a.ldo]) : 0.f;
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (nok && m0 + c + j < a.M) col[(size_t)j * a.ldo] = from_f<bf16>(xr[j] + round_st<bf16>(v[j] + bn));
         } else if (a.out_f32) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) {

@@ -449,7 +449,9 @@ __global__ void __launch_bounds__(NT) argmax_pass2(const float* pv, const int64_
 
 int argmax_parts(size_t rows, size_t n) {
   long long by_size = (long long)((n + 2047) / 2048);
-  long long by_sms = (2LL * num_sms() + (long long)rows - 1) / (long long)(rows ? rows : 1);
+  // enough CTAs to cover the machine several times over (the pass is a
+  // latency-bound scan: short per-thread chains matter more than CTA count)
+  long long by_sms = (8LL * num_sms() + (long long)rows - 1) / (long long)(rows ? rows : 1);
   long long p = by_size < by_sms ? by_size : by_sms;
   if (p > 256) p = 256;
   if (p < 1) p = 1;
