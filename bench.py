@@ -40,6 +40,7 @@ import synth  # noqa: E402
 METRIC = "decode tok/s (Qwen2-1.5B shape, bf16, B=1/64); achieved HBM GB/s vs peak"
 WORKLOAD = "qwen2-1.5b-b1-prompt512-decode128"
 WORKLOAD_B64 = "qwen2-1.5b-b64-ctx4096-decode32"
+WORKLOAD_LONG = "qwen2-1.5b-b1-prompt32768-decode64"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -362,6 +363,10 @@ def run_ours(args, dist: Dist):
     pk, pk_kind = peaks()
     hbm = float(pk["hbm_gbs"])
     gemms = None
+    long_line = None
+    if not args.no_long_prefill:
+        wl_long = synth.WORKLOADS[WORKLOAD_LONG]
+        long_line = long_prefill(shape, wl_long["seed"] + 100 * dist.rank, wl_long["prompt"])
     if not args.no_prefill_gemms:
         gemms = prefill_gemm_rates(shape, args.prefill_gemm_tokens, float(pk["bf16_tflops"]))
     gu_ms, gu_n = ktimes["gate_up"]
@@ -395,6 +400,7 @@ def run_ours(args, dist: Dist):
         "gpu_launches": kernels_per_step * args.steps,
         "kernels_per_step": kernels_per_step,
         "prefill": {"tokens": prompt_len, "ms": pre_ms, "tok_s": prompt_len / (pre_ms / 1e3)},
+        "prefill_long": long_line,
         "prefill_gemms": gemms and {"tokens_per_chunk": args.prefill_gemm_tokens,
                                     "peak_tflops": float(pk["bf16_tflops"]), "peak_kind": pk_kind,
                                     "kernel": "tc_gemm_kernel (tcgen05, TMEM)", "shapes": gemms},
@@ -437,6 +443,24 @@ def prefill_gemm_rates(shape, tokens: int, peak_tflops: float, reps: int = 10):
     return out
 
 
+def long_prefill(shape, seed: int, tokens: int):
+    """Prefill of one `tokens`-token prompt on a fresh batch-1 model (weights
+    drawn on the device), timed with CUDA events after one untimed run."""
+    import qwen2_decode_step_b200 as q2
+    m = q2.Model(shape, max_seq=tokens + 8, max_batch=1)
+    for key in shape.weight_shapes():
+        t = synth.weight(shape, key[0], key[1], seed, device="cuda")
+        m.load_weight(key[0], key[1], t)
+        del t
+    ids = synth.prompt_ids(shape, tokens, seed, device="cuda")
+    m.prefill(ids, [tokens])
+    m.reset_kv()
+    ms = cuda_time(lambda: m.prefill(ids, [tokens]), 1)
+    m.check_error()
+    m.close()
+    return {"workload": WORKLOAD_LONG, "tokens": tokens, "ms": ms, "tok_s": tokens / (ms / 1e3)}
+
+
 def cuda_time_b64(model, bufs, n):
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
@@ -458,6 +482,8 @@ def main():
     ap.add_argument("--no-b64", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill-gemms", action="store_true")
+    ap.add_argument("--no-long-prefill", action="store_true",
+                    help="skip the 32768-token prefill timing")
     ap.add_argument("--prefill-gemm-tokens", type=int, default=4096,
                     help="tokens of the prefill chunk whose linears are timed (the model's chunk size)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
