@@ -416,17 +416,9 @@ q2_status tc_gemm(void* out, int ldo, int out_dtype, int epi, const void* x, con
   a.out_f32 = out_dtype == Q2_F32;
   a.epi = epi;
   a.err = err;
-  // Token tile: the widest that fills the SMs' waves about as well as any
-  // (256 unless a narrower tile wastes at least 15 % less of the last wave).
-  int bn = M >= 256 ? 256 : (M >= 128 ? 128 : 64);
-  if (bn == 256) {
-    auto wave_eff = [&](int w) {
-      const long long t = (long long)((N + kBM - 1) / kBM) * ((M + w - 1) / w);
-      const long long waves = (t + num_sms() - 1) / num_sms();
-      return (double)t / (double)(waves * num_sms());
-    };
-    if (wave_eff(128) > wave_eff(256) + 0.15) bn = 128;
-  }
+  // Token tile: 256 wide from 256 tokens up (narrower tiles fill the last
+  // wave better but double the operand traffic per FLOP; measured slower).
+  const int bn = M >= 256 ? 256 : (M >= 128 ? 128 : 64);
   // Split K when the tiles alone would leave SMs idle (few output features,
   // few tokens): aim for one work item per SM, at least two k-blocks each,
   // within the workspace.
