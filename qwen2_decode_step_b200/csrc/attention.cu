@@ -235,7 +235,9 @@ __global__ void attn_combine_kernel(AttnRows a, int nsplit, const float* part_o,
 
 int attn_splits(int rows, int nkv, int max_keys) {
   long long ctas = (long long)rows * nkv;
-  long long want = (2LL * num_sms() + ctas - 1) / (ctas ? ctas : 1);
+  // as many splits as fit one wave of two CTAs per SM (a partial second wave
+  // would leave most SMs idle for its duration); at least one
+  long long want = (2LL * num_sms()) / (ctas ? ctas : 1);
   long long cap = (max_keys + kTK - 1) / kTK;
   if (cap > 64) cap = 64;
   if (want > cap) want = cap;
