@@ -1,0 +1,112 @@
+"""The batch-64 workload (Qwen2-1.5B shape, bf16, 64 sequences at 4096
+cached positions, N(0,1) cache) at full size, in the launch configuration
+the bench times: tcgen05 linears with M = 64 tokens (split-K for the 1536-
+and 2048-row projections) and the tensor-core decode attention (two splits
+per sequence and kv head).
+
+The oracle decodes sampled sequences one by one over the same cache:
+* layer by layer with teacher forcing (each layer's sampled rows fed the
+  oracle's input for that layer; rows are independent sequences), within the
+  per-layer bound;
+* the whole step free-running for sampled sequences, within the long-context
+  free-running bound (the oracle's own fp32-accumulation drift, doubled, as
+  measured at 32768 positions: an upper bound at 4096).
+"""
+import dataclasses
+
+import pytest
+import torch
+
+import oracle
+import qwen2_decode_step_b200 as q2
+import synth
+from tol import assert_layer_close
+
+pytestmark = pytest.mark.gpu
+
+WL = synth.WORKLOADS["qwen2-1.5b-b64-ctx4096-decode32"]
+SAMPLED = (0, 37, 63)
+
+
+@pytest.fixture(autouse=True)
+def _gpu(cuda_ok):
+    pass
+
+
+@pytest.fixture(scope="module")
+def b64():
+    shape = synth.QWEN2_1P5B
+    seed, past, B = WL["seed"], WL["past"], WL["batch"]
+    w = synth.model_weights(shape, seed, device="cuda")
+    wc = {k: t.cpu() for k, t in w.items()}
+    ids = synth.uniform_ids(B, shape.vocab, seed + 7)
+    return shape, seed, past, B, w, wc, ids
+
+
+def _fill_cache(model, shape, seed, past, B, layers, dst_layer=None):
+    """The N(0,1) cache of the workload for `layers`, written into `model`
+    (at dst_layer when given); returns the sampled sequences' K/V on the host."""
+    host = {}
+    for l in layers:
+        for b in range(B):
+            k, v = synth.kv_fill(shape, past, seed, l, b, device="cuda")
+            gk, gv = model.kv_cache(l if dst_layer is None else dst_layer, b)
+            gk[:, :past] = k.permute(1, 0, 2)
+            gv[:, :past] = v.permute(1, 0, 2)
+            if b in SAMPLED:
+                host[(l, b)] = (k.cpu(), v.cpu())
+    for b in range(B):
+        model.set_seq_len(b, past)
+    return host
+
+
+def test_batch64_decode_layerwise_teacher_forced(b64):
+    shape, seed, past, B, w, wc, ids = b64
+    one = dataclasses.replace(shape, n_layers=1)
+    g1 = q2.Model(one, max_seq=past + 8, max_batch=B)
+    g1.load({k: t for k, t in w.items() if k[1] == -1})
+    emb = wc[("embed", -1)]
+    x_ref = {b: oracle.embedding(ids[b:b + 1], emb) for b in SAMPLED}
+    x = oracle.embedding(ids, emb).cuda()  # all 64 rows (rows are independent sequences)
+    for l in range(shape.n_layers):
+        g1.load({(n, 0): t for (n, ll), t in w.items() if ll == l})
+        host = _fill_cache(g1, shape, seed, past, B, [l], dst_layer=0)
+        for b in SAMPLED:
+            x[b] = x_ref[b][0].cuda()
+        y = g1.forward_hidden(x)
+        om = oracle.OracleModel(one, max_seq=past + 8)
+        om.load({(n, 0): t for (n, ll), t in wc.items() if ll == l})
+        for b in SAMPLED:
+            ok, ov = om.kv(0, 0)
+            ok[:past] = host[(l, b)][0]
+            ov[:past] = host[(l, b)][1]
+            om.set_len(0, past)
+            y_ref = om.forward_hidden(0, x_ref[b])
+            assert_layer_close(y[b:b + 1], y_ref, f"layer {l} sequence {b}")
+            x_ref[b] = y_ref
+        del om
+        x = y
+
+
+def test_batch64_decode_step_free_running(b64):
+    shape, seed, past, B, w, wc, ids = b64
+    gm = q2.Model(shape, max_seq=past + 8, max_batch=B)
+    gm.load(w)
+    host = _fill_cache(gm, shape, seed, past, B, range(shape.n_layers))
+    nxt, lg = gm.decode_step(ids.cuda(), want_logits=True)
+    for b in SAMPLED:
+        om = oracle.OracleModel(shape, max_seq=past + 8)
+        om.load(wc)
+        for l in range(shape.n_layers):
+            ok, ov = om.kv(l, 0)
+            ok[:past] = host[(l, b)][0]
+            ov[:past] = host[(l, b)][1]
+        om.set_len(0, past)
+        _, lg_ref = om.forward(0, ids[b:b + 1])
+        g, r = lg[b].double().cpu(), lg_ref.double()
+        mx = float((g - r).abs().max())
+        cos = float(torch.nn.functional.cosine_similarity(g, r, dim=0))
+        assert mx <= 0.25 and cos >= 0.999, f"sequence {b}: max-abs {mx:.3e}, cosine {cos:.6f}"
+        del om
+    for b in range(B):
+        assert gm.get_seq_len(b) == past + 1
