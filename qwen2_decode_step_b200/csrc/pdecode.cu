@@ -290,8 +290,10 @@ __global__ void __launch_bounds__(kThreads, 1) pdecode_kernel(const PDecode p, c
   }
   __syncthreads();
 
-  const int NACC = RING + 1;  // row-group accumulators (see the producer)
-  const unsigned ARRIVALS = 2u * (unsigned)G;  // per phase: consumers and producer of every CTA
+  // Row-group accumulators: the producer issues a group's first stage only
+  // after the epilogue warp has read the group that last used its accumulator.
+  const int NACC = RING + 1;
+  const unsigned ARRIVALS = 2u * (unsigned)G;  // per phase: consumers and epilogue warp of every CTA
 
   // The last arrival of the last phase wraps up the step: the step's token
   // per sequence (argmax over the CTAs' partials) and the lengths.
@@ -567,9 +569,10 @@ __global__ void __launch_bounds__(kThreads, 1) pdecode_kernel(const PDecode p, c
   // terms in any order, those eight columns feed two MMAs directly (one column
   // permutation shared by both operands).  Each warp keeps its partial sums
   // of the group in its own slice of the group's accumulator (summing its kb
-  // column blocks in order); the last of the kC * kb contributions runs the
-  // epilogue, lane (r, m) adding the kC slices of row r, token m in warp
-  // order -- a fixed summation order, so every step is bit-reproducible.
+  // column blocks in order) and signals `posted` after the group's last
+  // column block; the epilogue warp then adds the kC slices of row r, token m
+  // in warp order -- a fixed summation order, so every step is
+  // bit-reproducible.
   auto gemv_phase = [&](const WPhase& wp) {
     const int K = wp.K, KT = wp.KT, kb = wp.kb, R = wp.R;
     const int ns = (wp.ge - wp.gb) * kb;

@@ -2,22 +2,26 @@
 // launch, one CTA per SM, runs a whole decode step (or the decoder layers
 // alone).
 //
-// Each CTA has a producer warp and kPConsumers consumer warps.  The producer
-// streams this CTA's share of every weight matrix of the step -- layer by
-// layer q/k/v, o, gate/up, down, then the lm_head -- through one TMA ring,
-// running ahead across phase boundaries as far as the ring allows.  The
-// consumers run the phases in order, separated by grid-wide counters:
-//   QKV(l)  RMSNorm prologue (layer 0: embedding gather), q/k/v rows,
-//           bias + RoPE, q out, K/V appended to the cache
-//   ATTN(l) split attention over the cache, partials out
-//   O(l)    prologue merges the attention partials; o rows, residual add
+// Each CTA has a producer warp, kPConsumers consumer warps and an epilogue
+// warp.  The producer streams this CTA's row groups of every weight matrix of
+// the step -- layer by layer q/k/v, o, gate/up, down, then the lm_head --
+// through one TMA ring (one bulk copy per weight row), running ahead across
+// phase boundaries as far as the ring allows and pulling later stages into
+// L2.  The consumers split each stage's columns and run the dot products on
+// the tensor cores (mma.sync), posting per-warp partial sums; the epilogue
+// warp finishes each row group (bias + RoPE + KV append, SwiGLU, residual
+// add, logits + argmax).  The phases run in order, separated by grid-wide
+// counters:
+//   QKV(l)  RMSNorm prologue (layer 0: embedding gather), q/k/v rows
+//   ATTN(l) split attention over the cache, splits merged by the last CTA
+//   O(l)    o rows, residual add
 //   GU(l)   RMSNorm prologue; gate/up row pairs, SwiGLU
 //   DOWN(l) down rows, residual add
-//   HEAD    final RMSNorm; lm_head rows, fp32 logits, argmax (the last CTA
-//           to arrive reduces), lengths advanced
-// Every grid-wide wait is bounded (a deadline on the global timer); a wait
-// that runs out sets bit 2 of the error word and the step carries on, so a
-// broken dependency can never hang the GPU.
+//   HEAD    final RMSNorm; lm_head rows, fp32 logits, argmax (the last arrival
+//           reduces the CTAs' partials), lengths advanced
+// Every wait is bounded (a deadline on the global timer); a wait that runs
+// out sets bit 1 of the error word and the step carries on, so a broken
+// dependency can never hang the GPU.
 #pragma once
 
 #include <cuda.h>
