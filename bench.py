@@ -10,8 +10,14 @@ Qwen2-1.5B shape, random-init bf16 weights, batch 1, a 512-token prompt of
 uniform random ids prefilled first (timed separately), then the timed decode
 steps (context 512 + warmup + steps).  Per step the kernels stream all
 3.09 GB of weights, far more than the 126 MB L2, so no L2 flush is needed.
-Extra keys report batch 64 at 4096 context (KV filled with N(0,1)), the
-prefill, per-kernel times and the CPU oracle baseline.
+Extra keys report batch 64 at 4096 context (`b64`, KV filled with N(0,1)),
+the 512-token prefill (`prefill`), the 32768-token prefill (`prefill_long`),
+the tcgen05 GEMM on the linears of a 4096-token prefill chunk
+(`prefill_gemms`, fraction of the measured bf16 peak), per-kernel times inside
+the decode step (`kernels_ms`), the roofline of the gate/up GEMV (`roofline`,
+with the DRAM traffic recorded under `profiles/` while its sources are
+unchanged), the host-buffer entry point end to end (`e2e`), SM clocks during
+the timed region (`clocks`) and the CPU oracle baseline (`cpu_baseline`).
 
 Multi-GPU: replicas (`--gpus N` under torchrun): every rank decodes its own
 sequences, no data-path collective; the time is the max over ranks.
