@@ -261,7 +261,6 @@ q2_status run_layers(q2_model* M, int T, int decode, int seq, int pos0, cudaStre
     a.nkv = m.n_kv_heads;
     a.hd = m.head_dim;
     a.scale = 1.0f / sqrtf((float)m.head_dim);
-    int nsplit;
     if (decode && M->fused && dt == Q2_BF16 &&
         dattn_mma_supported(m.n_heads, m.n_kv_heads, m.head_dim, decode_splits(M, T))) {
       // decode rows over the cache: the tensor-core attention
@@ -284,25 +283,25 @@ q2_status run_layers(q2_model* M, int T, int decode, int seq, int pos0, cudaStre
       d.scale = 1.0f / sqrtf((float)m.head_dim);
       d.err = M->d_err;
       TIMED(Q2_K_ATTN, launch_dattn_mma(d, M->kmap, M->vmap, st));
-      goto attention_done;
-    }
-    if (decode) {
-      a.base = 1;
-      a.row_step = 0;
-      a.lens = M->d_len;
-      a.seq_is_row = 1;
-      a.fixed_seq = 0;
-      nsplit = decode_splits(M, T);
     } else {
-      a.base = pos0 + 1;
-      a.row_step = 1;
-      a.lens = nullptr;
-      a.seq_is_row = 0;
-      a.fixed_seq = seq;
-      nsplit = attn_splits(T, m.n_kv_heads, pos0 + T);
+      int nsplit;
+      if (decode) {
+        a.base = 1;
+        a.row_step = 0;
+        a.lens = M->d_len;
+        a.seq_is_row = 1;
+        a.fixed_seq = 0;
+        nsplit = decode_splits(M, T);
+      } else {
+        a.base = pos0 + 1;
+        a.row_step = 1;
+        a.lens = nullptr;
+        a.seq_is_row = 0;
+        a.fixed_seq = seq;
+        nsplit = attn_splits(T, m.n_kv_heads, pos0 + T);
+      }
+      TIMED(Q2_K_ATTN, launch_attention(a, nsplit, M->attn_scratch, dt, st, pdl));
     }
-    TIMED(Q2_K_ATTN, launch_attention(a, nsplit, M->attn_scratch, dt, st, pdl));
-  attention_done:
 
     if (tc) {
       TIMED(Q2_K_O, tc_gemm(M->x, H, Q2_BF16, TC_EPI_RESID, M->att, w.wo, nullptr, T, H, M->qd, st, M->tc_ws,
