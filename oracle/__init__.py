@@ -24,7 +24,10 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "oracle.c")
 _HDR = os.path.join(_HERE, "oracle.h")
 _BUILD = os.path.join(_HERE, "_build")
-_LIB_PATH = os.path.join(_BUILD, "liboracle.so")
+# ORACLE_FP32_ACCUMULATION=1 in the environment selects the fp32-accumulating
+# copy (a tolerance-derivation tool, see oracle/drift.py), never the default.
+_F32ACC = os.environ.get("ORACLE_FP32_ACCUMULATION") == "1"
+_LIB_PATH = os.path.join(_BUILD, "liboracle_f32acc.so" if _F32ACC else "liboracle.so")
 
 F32, BF16 = 0, 1
 _CODE = {torch.float32: F32, torch.bfloat16: BF16}
@@ -50,7 +53,7 @@ def build(force: bool = False) -> str:
     if force or stale:
         tmp = _LIB_PATH + f".tmp{os.getpid()}"
         cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math", "-ffp-contract=off",
-               "-o", tmp, _SRC, "-lm"]
+               *(["-DORACLE_FP32_ACCUMULATION"] if _F32ACC else []), "-o", tmp, _SRC, "-lm"]
         subprocess.run(cmd, check=True)
         os.replace(tmp, _LIB_PATH)
     return _LIB_PATH

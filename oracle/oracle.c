@@ -10,6 +10,18 @@
  */
 #include "oracle.h"
 
+/* The accumulator of the linear and of attention's probability-weighted sum
+ * of V: double.  Building with -DORACLE_FP32_ACCUMULATION makes it float --
+ * not an oracle, but a copy of it with the rounding behaviour of fp32
+ * accumulation, used only to measure how far that alone moves the model's
+ * logits (oracle/drift.py), from which the free-running tolerances are
+ * derived. */
+#ifdef ORACLE_FP32_ACCUMULATION
+typedef float oracle_acc_t;
+#else
+typedef double oracle_acc_t;
+#endif
+
 #include <math.h>
 #include <stdlib.h>
 #include <string.h>
@@ -143,13 +155,13 @@ int oracle_linear(void* y, const void* x, const void* w, const void* b, size_t M
   for (size_t m = 0; m < M; ++m) {
     for (size_t k = 0; k < K; ++k) xs[k] = ld(x, m * K + k, dtype);
     for (size_t n = 0; n < N; ++n) {
-      double acc = 0.0;
+      oracle_acc_t acc = 0.0;
       if (dtype == ORACLE_BF16) {
         const uint16_t* wr = (const uint16_t*)w + n * K;
-        for (size_t k = 0; k < K; ++k) acc += xs[k] * oracle_bf16_to_double(wr[k]);
+        for (size_t k = 0; k < K; ++k) acc += (oracle_acc_t)xs[k] * (oracle_acc_t)oracle_bf16_to_double(wr[k]);
       } else {
         const float* wr = (const float*)w + n * K;
-        for (size_t k = 0; k < K; ++k) acc += xs[k] * (double)wr[k];
+        for (size_t k = 0; k < K; ++k) acc += (oracle_acc_t)xs[k] * (oracle_acc_t)wr[k];
       }
       if (b) acc += ld(b, n, dtype);
       st(y, m * N + n, acc, out_dtype);
@@ -247,8 +259,8 @@ int oracle_self_attention(void* out, const void* q, const void* k, const void* v
       }
       if (!(fabs(mass - 1.0) <= 1e-12)) rc = ORACLE_ECHECK;
       for (size_t d = 0; d < hd; ++d) {
-        double acc = 0.0;
-        for (size_t j = 0; j <= last; ++j) acc += p[j] * ld(v, (j * nkv + g) * hd + d, dtype);
+        oracle_acc_t acc = 0.0;
+        for (size_t j = 0; j <= last; ++j) acc += (oracle_acc_t)p[j] * (oracle_acc_t)ld(v, (j * nkv + g) * hd + d, dtype);
         st(out, qb + d, acc, dtype);
       }
     }

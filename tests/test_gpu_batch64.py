@@ -9,18 +9,17 @@ The oracle decodes sampled sequences one by one over the same cache:
   oracle's input for that layer; rows are independent sequences), within the
   per-layer bound;
 * the whole step free-running for sampled sequences, within the long-context
-  free-running bound (the oracle's own fp32-accumulation drift, doubled, as
-  measured at 32768 positions: an upper bound at 4096).
+  free-running bound (twice the oracle's own fp32-accumulation drift at
+  32768 positions, an upper bound for 4096).
 """
 import dataclasses
 
 import pytest
-import torch
 
 import oracle
 import qwen2_decode_step_b200 as q2
 import synth
-from tol import assert_layer_close
+from tol import assert_bf16_logits_long_context, assert_layer_close
 
 pytestmark = pytest.mark.gpu
 
@@ -103,10 +102,7 @@ def test_batch64_decode_step_free_running(b64):
             ov[:past] = host[(l, b)][1]
         om.set_len(0, past)
         _, lg_ref = om.forward(0, ids[b:b + 1])
-        g, r = lg[b].double().cpu(), lg_ref.double()
-        mx = float((g - r).abs().max())
-        cos = float(torch.nn.functional.cosine_similarity(g, r, dim=0))
-        assert mx <= 0.25 and cos >= 0.999, f"sequence {b}: max-abs {mx:.3e}, cosine {cos:.6f}"
+        assert_bf16_logits_long_context(lg[b], lg_ref, f"sequence {b}")
         del om
     for b in range(B):
         assert gm.get_seq_len(b) == past + 1

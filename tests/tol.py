@@ -70,6 +70,23 @@ def assert_layer_close(got: torch.Tensor, ref: torch.Tensor, what: str = ""):
 FREE_RUNNING_MAXABS = 0.15
 
 
+# Long context (4096-32768 cached positions): the oracle's own drift when it
+# accumulates in fp32 (python -m oracle.drift cache --context 32768) is
+# max-abs 0.115, cosine 0.999429; a GPU path accumulating in fp32 is held to
+# twice that drift.
+LONG_FREE_MAXABS = 0.25
+LONG_FREE_COS = 0.9988
+
+
+def assert_bf16_logits_long_context(got: torch.Tensor, ref: torch.Tensor, what: str = ""):
+    g = got.detach().double().cpu().reshape(-1)
+    r = ref.detach().double().cpu().reshape(-1)
+    mx = float((g - r).abs().max())
+    cos = float(torch.nn.functional.cosine_similarity(g, r, dim=0))
+    assert mx <= LONG_FREE_MAXABS and cos >= LONG_FREE_COS, f"{what}: max-abs {mx:.3e}, cosine {cos:.6f}"
+    return mx, cos
+
+
 def assert_bf16_logits_free_running(got: torch.Tensor, ref: torch.Tensor, what: str = ""):
     g = got.detach().double().cpu().reshape(-1)
     r = ref.detach().double().cpu().reshape(-1)
