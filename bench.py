@@ -12,8 +12,9 @@ steps (context 512 + warmup + steps).  Per step the kernels stream all
 3.09 GB of weights, far more than the 126 MB L2, so no L2 flush is needed.
 Extra keys report batch 64 at 4096 context (`b64`, KV filled with N(0,1)),
 the 512-token prefill (`prefill`), the 32768-token prefill (`prefill_long`),
-the tcgen05 GEMM on the linears of a 4096-token prefill chunk
-(`prefill_gemms`, fraction of the measured bf16 peak), per-kernel times inside
+the tcgen05 GEMM on the prefill linears at 4096 tokens (the model's prefill
+chunk) and 32768 tokens (`prefill_gemms`, fraction of the measured bf16
+peak), per-kernel times inside
 the decode step (`kernels_ms`), the roofline of the gate/up GEMV (`roofline`,
 with the DRAM traffic recorded under `profiles/` while its sources are
 unchanged), the host-buffer entry point end to end (`e2e`), SM clocks during
@@ -374,7 +375,8 @@ def run_ours(args, dist: Dist):
         wl_long = synth.WORKLOADS[WORKLOAD_LONG]
         long_line = long_prefill(shape, wl_long["seed"] + 100 * dist.rank, wl_long["prompt"])
     if not args.no_prefill_gemms:
-        gemms = prefill_gemm_rates(shape, args.prefill_gemm_tokens, float(pk["bf16_tflops"]))
+        gemms = {str(t): prefill_gemm_rates(shape, t, float(pk["bf16_tflops"]))
+                 for t in (int(x) for x in args.prefill_gemm_tokens.split(","))}
     gu_ms, gu_n = ktimes["gate_up"]
     gu_bytes = 2 * shape.intermediate * shape.hidden * 2 + shape.hidden * 2 + 2 * shape.intermediate * 2
     achieved = gu_bytes / (gu_ms / 1e3) / 1e9 if gu_ms > 0 else None
@@ -407,9 +409,9 @@ def run_ours(args, dist: Dist):
         "kernels_per_step": kernels_per_step,
         "prefill": {"tokens": prompt_len, "ms": pre_ms, "tok_s": prompt_len / (pre_ms / 1e3)},
         "prefill_long": long_line,
-        "prefill_gemms": gemms and {"tokens_per_chunk": args.prefill_gemm_tokens,
+        "prefill_gemms": gemms and {"tokens": args.prefill_gemm_tokens,
                                     "peak_tflops": float(pk["bf16_tflops"]), "peak_kind": pk_kind,
-                                    "kernel": "tc_gemm_kernel (tcgen05, TMEM)", "shapes": gemms},
+                                    "kernel": "tc_gemm_kernel (tcgen05, TMEM)", "by_tokens": gemms},
         "e2e": {"value": 1 * dist.world / (e2e_ms / 1e3), "unit": "tok/s", "h2d_bytes_per_step": 8,
                 "d2h_bytes_per_step": 8, "ms_per_step": e2e_ms,
                 "api": "q2_model_decode_step_host (pinned host ids -> host next)"},
@@ -490,8 +492,9 @@ def main():
     ap.add_argument("--no-prefill-gemms", action="store_true")
     ap.add_argument("--no-long-prefill", action="store_true",
                     help="skip the 32768-token prefill timing")
-    ap.add_argument("--prefill-gemm-tokens", type=int, default=4096,
-                    help="tokens of the prefill chunk whose linears are timed (the model's chunk size)")
+    ap.add_argument("--prefill-gemm-tokens", default="4096,32768",
+                    help="token counts at which the prefill linears are timed: the model's prefill "
+                         "chunk (4096) and the whole 32768-token prompt as one product")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     args = ap.parse_args()
     if args.warmup < 3:
