@@ -30,8 +30,9 @@
  * - Sizes are element counts unless named *_bytes.
  * - Argument checks that need no device access happen before any launch and
  *   leave outputs untouched.  Errors that only the GPU can see (a token id
- *   outside the vocabulary) are recorded in a device-side flag and reported
- *   by q2_check_device_error() / q2_model_check_error().
+ *   outside the vocabulary; a bounded wait inside a kernel that ran out) are
+ *   recorded in a device-side flag and reported by q2_check_device_error() /
+ *   q2_model_check_error().
  */
 #ifndef Q2_H
 #define Q2_H
@@ -52,7 +53,10 @@ typedef enum q2_status {
   Q2_ERR_INDEX = 5,       /* a kernel saw a token id outside [0, vocab) */
   Q2_ERR_CUDA = 6,        /* a CUDA runtime call failed (message in q2_last_error) */
   Q2_ERR_OOM = 7,         /* device allocation failed */
-  Q2_ERR_STATE = 8        /* call not valid in the object's current state */
+  Q2_ERR_STATE = 8,       /* call not valid in the object's current state */
+  Q2_ERR_TIMEOUT = 9      /* a bounded device-side wait ran out: a pipeline or grid-phase
+                             dependency never arrived; results since the last check are
+                             undefined (reported by the check functions) */
 } q2_status;
 
 typedef enum q2_dtype { Q2_F32 = 0, Q2_BF16 = 1 } q2_dtype;
@@ -62,10 +66,17 @@ const char* q2_last_error(void);
 /* Library version string, e.g. "q2 0.1 sm_100a". */
 const char* q2_version(void);
 
-/* Synchronises `stream`, then returns Q2_ERR_INDEX if any per-operator kernel
- * on the current device recorded an out-of-range id since the last check
- * (and clears the record), else Q2_OK. */
+/* Synchronises `stream`, then reports what the per-operator kernels on the
+ * current device recorded since the last check, and clears the record:
+ * Q2_ERR_TIMEOUT if a bounded wait inside a kernel ran out (the tcgen05 GEMM
+ * behind q2_linear), else Q2_ERR_INDEX if a kernel saw a token id outside
+ * the vocabulary, else Q2_OK. */
 q2_status q2_check_device_error(void* stream);
+
+/* Test hook: ORs `bits` (1: out-of-range id, 2: wait ran out) into the
+ * operators' device error word of the current device, as a kernel would.
+ * Synchronises. */
+q2_status q2_test_raise_device_error(int bits, void* stream);
 
 /* ======================================================================== */
 /* Operators (report section 3.2, third layer).  Device pointers, caller-   */
@@ -298,29 +309,59 @@ q2_status q2_model_get_seq_len(const q2_model* model, int seq, int* len);
  * at element (g * max_seq + p) * hd).  The model keeps ownership. */
 q2_status q2_model_kv_cache(q2_model* model, int layer, int seq, void** k, void** v);
 
-/* Synchronises `stream`, then returns Q2_ERR_INDEX if a model kernel saw a
- * token id outside the vocabulary since the last check (and clears the
- * record), else Q2_OK. */
+/* Synchronises `stream`, then reports what the model's kernels recorded since
+ * the last check, and clears the record: Q2_ERR_TIMEOUT if a bounded
+ * device-side wait ran out (every wait in the decode kernels, the persistent
+ * and streaming steps and the tcgen05 GEMM gives up after a deadline instead
+ * of hanging; the results since the last check are then undefined), else
+ * Q2_ERR_INDEX if a kernel saw a token id outside the vocabulary, else Q2_OK. */
 q2_status q2_model_check_error(q2_model* model, void* stream);
+
+/* Test hook: ORs `bits` (1: out-of-range id, 2: wait ran out) into the model's
+ * device error word, as a kernel would.  Synchronises. */
+q2_status q2_test_model_raise_error(q2_model* model, int bits, void* stream);
+
+/* Profiling hook of the batch-1 streaming step: runs one step on ids_dev[0]
+ * (eager launch, not a graph) with per-CTA timestamps of the global timer and
+ * copies them to `out` (host, n >= (5 * n_layers + 1) * grid * 4 words): for
+ * phase p and CTA c, out[(p * grid + c) * 4 + k] with k = 0 phase entered,
+ * 1 previous phase seen complete, 2 phase work done, 3 arrival; `grid` gets
+ * the CTA count.  The model's lengths are restored afterwards (the K/V rows
+ * of the traced position are written).  Synchronises. */
+q2_status q2_test_trace_stream_step(q2_model* model, const int64_t* ids_dev, unsigned long long* out,
+                                    size_t n, int* grid, void* stream);
+
+/* Test hook for the waits of the batch-1 streaming step: with phase >= 0 the
+ * grid counter of that phase (phases of layer l are 5l .. 5l+4: q/k/v,
+ * attention, o, gate/up, down; 5 * n_layers is the lm_head) needs one more
+ * arrival than the grid makes, so every CTA's wait on it runs out, and every
+ * wait is bounded by `deadline_ns` instead of 200 ms; the step then carries
+ * on and q2_model_check_error reports Q2_ERR_TIMEOUT.  phase = -1 restores
+ * the defaults.  Drops the captured decode graphs.  Not for production use. */
+q2_status q2_test_set_wait_fault(q2_model* model, int phase, unsigned long long deadline_ns);
 
 /* Turns CUDA-graph capture of decode steps on (default) or off (eager
  * launches, for debugging and per-kernel timing). */
 q2_status q2_model_set_graphs(q2_model* model, int enable);
 
 /* Decode-step implementation for bf16 models at batch <= 4:
- * Q2_PATH_AUTO (default: the persistent kernel for 2 <= batch <= 4, the fused
- * per-layer kernels at batch 1, where the shapes allow),
+ * Q2_PATH_AUTO (default: the streaming step at batch 1, the persistent kernel
+ * for 2 <= batch <= 4, where the shapes allow),
  * Q2_PATH_PERSISTENT (one cooperative launch per step: every CTA streams its
  * share of all weights through one TMA ring while the phases of the step run
  * between grid-wide counters), Q2_PATH_KERNELS (five fused kernels per layer
  * chained by programmatic dependent launch), Q2_PATH_GENERIC (one kernel per
- * operator).  Larger batches and fp32 models always take the generic path.
+ * operator), Q2_PATH_STREAM (batch 1 only: one cooperative launch per step
+ * whose producer warps stream the weights of every phase ahead of the
+ * phases, while the consumer warps run the phases between grid-wide
+ * counters).  Larger batches and fp32 models always take the generic path.
  * Q2_ERR_STATE if the requested path is not available for this model. */
 typedef enum q2_path {
   Q2_PATH_AUTO = 0,
   Q2_PATH_PERSISTENT = 1,
   Q2_PATH_KERNELS = 2,
-  Q2_PATH_GENERIC = 3
+  Q2_PATH_GENERIC = 3,
+  Q2_PATH_STREAM = 4
 } q2_path;
 q2_status q2_model_set_decode_path(q2_model* model, int path);
 

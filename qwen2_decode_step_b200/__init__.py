@@ -19,7 +19,7 @@ import torch
 
 __all__ = [
     "Q2Error", "lib", "q2_version", "q2_check_device_error", "q2_add", "q2_argmax",
-    "q2_argmax_noalloc", "q2_embedding",
+    "q2_argmax_noalloc", "q2_embedding", "q2_test_raise_device_error",
     "q2_linear", "q2_test_tc_gemm", "q2_rms_norm", "q2_add_rms_norm", "q2_rope", "q2_self_attention", "q2_swiglu",
     "q2_rearrange", "Model", "W_KIND", "STATUS", "KCLASS",
 ]
@@ -29,7 +29,7 @@ LIB_PATH = os.path.join(_PKG, "lib", "libq2.so")
 
 STATUS = {0: "Q2_OK", 1: "Q2_ERR_INVALID_ARG", 2: "Q2_ERR_DTYPE", 3: "Q2_ERR_SHAPE",
           4: "Q2_ERR_CAPACITY", 5: "Q2_ERR_INDEX", 6: "Q2_ERR_CUDA", 7: "Q2_ERR_OOM",
-          8: "Q2_ERR_STATE"}
+          8: "Q2_ERR_STATE", 9: "Q2_ERR_TIMEOUT"}
 F32, BF16 = 0, 1
 _DT = {torch.float32: F32, torch.bfloat16: BF16}
 W_KIND = {"embed": 0, "lm_head": 1, "final_norm": 2, "in_norm": 3, "q_w": 4, "q_b": 5, "k_w": 6,
@@ -84,11 +84,15 @@ _SIGS = {
     "q2_model_prefill_hidden": [_VP, _I, _VP, _I, _VP, _VP],
     "q2_model_head": [_VP, _VP, _I, _VP, _VP, _VP],
     "q2_model_set_decode_path": [_VP, _I],
+    "q2_test_raise_device_error": [_I, _VP],
+    "q2_test_model_raise_error": [_VP, _I, _VP],
+    "q2_test_set_wait_fault": [_VP, _I, ctypes.c_ulonglong],
+    "q2_test_trace_stream_step": [_VP, _VP, _VP, _SZ, ctypes.POINTER(_I), _VP],
 }
 
 KCLASS = ["embed", "norm", "qkv", "rope_kv", "attn", "o", "gate_up", "swiglu", "down", "lm_head",
           "argmax", "other", "step"]
-PATH = {"auto": 0, "persistent": 1, "kernels": 2, "generic": 3}
+PATH = {"auto": 0, "persistent": 1, "kernels": 2, "generic": 3, "stream": 4}
 
 _lib = None
 
@@ -152,6 +156,11 @@ def q2_version() -> str:
 
 def q2_check_device_error() -> None:
     _call("q2_check_device_error", _stream())
+
+
+def q2_test_raise_device_error(bits: int) -> None:
+    """Test hook: OR `bits` into the operators' device error word."""
+    _call("q2_test_raise_device_error", bits, _stream())
 
 
 def q2_add(c, a, b):
@@ -388,11 +397,32 @@ class Model:
     def check_error(self):
         _call("q2_model_check_error", self._h, _stream())
 
+    def test_raise_error(self, bits: int):
+        """Test hook: OR `bits` into the model's device error word (q2_test_model_raise_error)."""
+        _call("q2_test_model_raise_error", self._h, bits, _stream())
+
+    def test_set_wait_fault(self, phase: int, deadline_ns: int = 200_000_000):
+        """Test hook: make one phase's grid counter of the streaming step
+        unreachable, with every wait bounded by deadline_ns (q2_test_set_wait_fault)."""
+        _call("q2_test_set_wait_fault", self._h, phase, deadline_ns)
+
+    def trace_stream_step(self, ids: torch.Tensor):
+        """Profiling hook: per-CTA timestamps of one streaming step,
+        [phases, grid, 4] int64 ns (q2_test_trace_stream_step)."""
+        import numpy as np
+        n = (5 * self.shape.n_layers + 1) * 160 * 4
+        buf = np.zeros(n, dtype=np.uint64)
+        g = ctypes.c_int()
+        _dense(ids)
+        _call("q2_test_trace_stream_step", self._h, _p(ids), buf.ctypes.data, n, ctypes.byref(g), _stream())
+        G = g.value
+        return torch.from_numpy(buf[: (5 * self.shape.n_layers + 1) * G * 4].astype(np.int64)).view(-1, G, 4)
+
     def set_graphs(self, enable: bool):
         _call("q2_model_set_graphs", self._h, 1 if enable else 0)
 
     def set_decode_path(self, path: str):
-        """'auto' | 'persistent' | 'kernels' | 'generic' (q2_model_set_decode_path)."""
+        """'auto' | 'persistent' | 'kernels' | 'generic' | 'stream' (q2_model_set_decode_path)."""
         _call("q2_model_set_decode_path", self._h, PATH[path])
 
     def time_kernels(self, ids: torch.Tensor, steps: int):

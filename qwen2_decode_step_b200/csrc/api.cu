@@ -43,6 +43,19 @@ int* op_error_flag() {
   return static_cast<int*>(p);
 }
 
+q2_status device_error_status(int bits, const char* who) {
+  std::string msg = std::string(who) + ": ";
+  if (bits & kErrTimeout) {
+    msg += "a bounded device-side wait ran out (a pipeline or grid-phase dependency never "
+           "arrived); the results of the calls since the last check are undefined";
+    if (bits & kErrIndex) msg += "; a kernel also saw a token id outside [0, vocab)";
+    set_error(msg);
+    return Q2_ERR_TIMEOUT;
+  }
+  set_error(msg + "a kernel saw a token id outside [0, vocab)");
+  return Q2_ERR_INDEX;
+}
+
 int num_sms() {
   static std::mutex mu;
   static std::map<int, int> cache;
@@ -82,9 +95,24 @@ q2_status q2_check_device_error(void* stream) {
   if (v) {
     int zero = 0;
     Q2_CUDA_TRY(cudaMemcpy(flag, &zero, sizeof zero, cudaMemcpyHostToDevice));
-    set_error("a kernel saw a token id outside [0, vocab)");
-    return Q2_ERR_INDEX;
+    return device_error_status(v, "check_device_error");
   }
+  return Q2_OK;
+}
+
+q2_status q2_test_raise_device_error(int bits, void* stream) {
+  clear_error();
+  Q2_CHECK_ARG(bits > 0 && bits <= (kErrIndex | kErrTimeout), Q2_ERR_INVALID_ARG,
+               "test_raise_device_error: bits must be 1, 2 or 3");
+  int* flag = op_error_flag();
+  Q2_CHECK_ARG(flag, Q2_ERR_CUDA, "cannot resolve the device error flag");
+  cudaStream_t st = as_stream(stream);
+  int cur = 0;
+  Q2_CUDA_TRY(cudaMemcpyAsync(&cur, flag, sizeof cur, cudaMemcpyDeviceToHost, st));
+  Q2_CUDA_TRY(cudaStreamSynchronize(st));
+  cur |= bits;
+  Q2_CUDA_TRY(cudaMemcpyAsync(flag, &cur, sizeof cur, cudaMemcpyHostToDevice, st));
+  Q2_CUDA_TRY(cudaStreamSynchronize(st));
   return Q2_OK;
 }
 
@@ -145,9 +173,11 @@ q2_status q2_test_tc_gemm(void* out, size_t ldo, int out_dtype, int epilogue, co
       return Q2_ERR_OOM;
     }
   }
+  int* flag = op_error_flag();
+  Q2_CHECK_ARG(flag, Q2_ERR_CUDA, "cannot resolve the device error flag");
   q2_status s = tc_gemm(out, (int)ldo, out_dtype, epilogue, x, w, bias, (int)M, (int)N, (int)K, st,
-                        ws, ws_bytes);
-  if (s == Q2_OK) s = tc_check_error(st);
+                        flag, ws, ws_bytes);
+  if (s == Q2_OK) s = q2_check_device_error(stream);
   if (ws) {
     cudaStreamSynchronize(st);
     cudaFree(ws);

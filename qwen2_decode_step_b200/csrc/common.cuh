@@ -47,9 +47,19 @@ q2_status launch_status(const char* what);
 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
-// Library-wide device error word of the per-operator kernels (bit 0: an id
-// outside the vocabulary).  One per device that loads the library.
+// Library-wide device error word of the per-operator kernels.  One per device
+// that loads the library.  Every error word (this one and each model's) uses
+// the same bits: value 1 = a token id outside [0, vocab); value 2 = a
+// bounded device-side wait ran out (a pipeline or grid-phase dependency that
+// never arrived).
 int* op_error_flag();
+constexpr int kErrIndex = 1;
+constexpr int kErrTimeout = 2;
+
+// The status (and message) of a nonzero error word: Q2_ERR_TIMEOUT if a wait
+// ran out (it takes precedence: the results are undefined), else
+// Q2_ERR_INDEX.  `who` prefixes the message.
+q2_status device_error_status(int bits, const char* who);
 
 // ------------------------------------------------------------ storage types
 template <typename T>

@@ -372,15 +372,6 @@ q2_status tc_launch(const CUtensorMap& tw, const CUtensorMap& tx, const TcArgs& 
   return Q2_OK;
 }
 
-// One sticky device word per device for "a pipeline wait ran out" (a static
-// symbol: nothing is allocated, so launches may be captured in CUDA graphs).
-__device__ int g_tc_err;
-
-int* tc_err_flag() {
-  void* p = nullptr;
-  return cudaGetSymbolAddress(&p, g_tc_err) == cudaSuccess ? static_cast<int*>(p) : nullptr;
-}
-
 }  // namespace
 
 bool tc_linear_supported(int M, int N, int K, const void* out, const void* in, const void* w) {
@@ -391,7 +382,8 @@ bool tc_linear_supported(int M, int N, int K, const void* out, const void* in, c
 }
 
 q2_status tc_gemm(void* out, int ldo, int out_dtype, int epi, const void* x, const void* w,
-                  const void* bias, int M, int N, int K, cudaStream_t st, float* ws, size_t ws_bytes) {
+                  const void* bias, int M, int N, int K, cudaStream_t st, int* err, float* ws,
+                  size_t ws_bytes) {
   if (M <= 0 || N <= 0) return Q2_OK;
   if (K % 8 != 0 || (reinterpret_cast<uintptr_t>(x) & 15) || (reinterpret_cast<uintptr_t>(w) & 15)) {
     set_error("tcgen05 gemm: K must be a multiple of 8 and operands 16-byte aligned");
@@ -401,10 +393,9 @@ q2_status tc_gemm(void* out, int ldo, int out_dtype, int epi, const void* x, con
     set_error("tcgen05 gemm: the SwiGLU epilogue needs an even N and a bf16 output");
     return Q2_ERR_INVALID_ARG;
   }
-  int* err = tc_err_flag();
   if (!err) {
-    set_error("tcgen05 gemm: no error flag");
-    return Q2_ERR_OOM;
+    set_error("tcgen05 gemm: no error word");
+    return Q2_ERR_INVALID_ARG;
   }
   TcArgs a;
   a.M = M;
@@ -442,26 +433,10 @@ q2_status tc_gemm(void* out, int ldo, int out_dtype, int epi, const void* x, con
   return tc_launch<64, 8>(tw, tx, a, st);
 }
 
-q2_status tc_check_error(cudaStream_t st) {
-  int* err = tc_err_flag();
-  if (!err) return Q2_OK;
-  int h = 0;
-  Q2_CUDA_TRY(cudaMemcpyAsync(&h, err, sizeof(int), cudaMemcpyDeviceToHost, st));
-  Q2_CUDA_TRY(cudaStreamSynchronize(st));
-  if (h) {
-    const int zero = 0;
-    cudaMemcpyAsync(err, &zero, sizeof(int), cudaMemcpyHostToDevice, st);
-    cudaStreamSynchronize(st);
-    set_error("tcgen05 gemm: a pipeline wait ran out");
-    return Q2_ERR_CUDA;
-  }
-  return Q2_OK;
-}
-
 q2_status tc_linear(void* out, const void* in, const void* w, const void* bias, int M, int N, int K,
                     int out_dtype, cudaStream_t st, bool pdl) {
   (void)pdl;
-  return tc_gemm(out, N, out_dtype, TC_EPI_PLAIN, in, w, bias, M, N, K, st, nullptr, 0);
+  return tc_gemm(out, N, out_dtype, TC_EPI_PLAIN, in, w, bias, M, N, K, st, op_error_flag(), nullptr, 0);
 }
 
 }  // namespace q2

@@ -18,16 +18,17 @@ enum { TC_EPI_PLAIN = 0, TC_EPI_SWIGLU = 1, TC_EPI_RESID = 2 };
 // N >= 128 features, K a multiple of 8, operands 16-byte aligned).
 bool tc_linear_supported(int M, int N, int K, const void* out, const void* in, const void* w);
 // out[M, N] (out_dtype) = in[M, K] . w[N, K]^T (+ bias[N]), bf16 operands.
+// A pipeline wait that runs out sets value 2 in the operators' error word.
 q2_status tc_linear(void* out, const void* in, const void* w, const void* bias, int M, int N, int K,
                     int out_dtype, cudaStream_t st, bool pdl);
 // The general form: output row stride `ldo` (elements) and an epilogue.  With
 // a workspace (fp32, `ws_bytes`), a product with fewer tiles than SMs splits
 // K across CTAs; the partial sums are added in a fixed order by a second
-// kernel, so results do not depend on scheduling.
+// kernel, so results do not depend on scheduling.  A pipeline wait that runs
+// out (a deadline on the global timer) sets value 2 in the device word `err`
+// (the caller's error word: the model's, or the operators').
 q2_status tc_gemm(void* out, int ldo, int out_dtype, int epi, const void* x, const void* w,
-                  const void* bias, int M, int N, int K, cudaStream_t st, float* ws = nullptr,
-                  size_t ws_bytes = 0);
-// Q2_ERR_CUDA (synchronising) if a pipeline wait in any tcgen05 GEMM ran out.
-q2_status tc_check_error(cudaStream_t st);
+                  const void* bias, int M, int N, int K, cudaStream_t st, int* err,
+                  float* ws = nullptr, size_t ws_bytes = 0);
 
 }  // namespace q2

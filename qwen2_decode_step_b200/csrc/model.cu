@@ -12,6 +12,7 @@
 // RMSNorm -> lm_head (fp32 logits) -> argmax.
 #include <math.h>
 
+#include <algorithm>
 #include <map>
 #include <vector>
 
@@ -20,6 +21,7 @@
 #include "kernels.h"
 #include "gemm_tc.h"
 #include "pdecode.h"
+#include "sdecode.h"
 #include <cstdlib>
 #include "tma.h"
 
@@ -85,6 +87,11 @@ struct q2_model {
   void* abuf = nullptr;
   bool fused = false;              // bf16 and the fused decode kernels support the shapes
   bool persistent = false;         // ... and the persistent decode kernel does too
+  bool streaming = false;          // ... and the batch-1 streaming step does too
+  int sd_ring = 0;                 // streaming step: weight ring slots (Q2_SDECODE_RING overrides)
+  int sd_l2_ahead = 0;             // streaming step: slots pulled into L2 ahead of the ring
+  unsigned long long wait_ns = 200ull * 1000 * 1000;  // bound of every device-side wait
+  int stall_phase = -1;            // test hook: a phase counter that never completes
   int path = Q2_PATH_AUTO;
   // Weight stages each CTA of the persistent step pulls into L2 ahead of its
   // shared-memory ring (Q2_PDECODE_L2_AHEAD overrides; 0 turns it off).
@@ -240,7 +247,7 @@ q2_status run_layers(q2_model* M, int T, int decode, int seq, int pos0, cudaStre
       TIMED(Q2_K_NORM, launch_add_rms_norm(M->x, nullptr, M->h, w.in_norm, T, H, m.eps, dt, st, pdl));
     if (tc)
       TIMED(Q2_K_QKV, tc_gemm(M->qkv, M->qkvd, Q2_BF16, TC_EPI_PLAIN, M->h, w.wqkv, w.bqkv, T, M->qkvd, H,
-                              st, M->tc_ws, M->tc_ws_bytes));
+                              st, M->d_err, M->tc_ws, M->tc_ws_bytes));
     else
       TIMED(Q2_K_QKV, launch_linear(M->qkv, M->h, w.wqkv, w.bqkv, T, M->qkvd, H, dt, dt, st, pdl));
     TIMED(Q2_K_ROPE_KV, launch_rope_kv(M, l, T, M->d_len, decode, seq, pos0, st, pdl));
@@ -304,12 +311,12 @@ q2_status run_layers(q2_model* M, int T, int decode, int seq, int pos0, cudaStre
     }
 
     if (tc) {
-      TIMED(Q2_K_O, tc_gemm(M->x, H, Q2_BF16, TC_EPI_RESID, M->att, w.wo, nullptr, T, H, M->qd, st, M->tc_ws,
+      TIMED(Q2_K_O, tc_gemm(M->x, H, Q2_BF16, TC_EPI_RESID, M->att, w.wo, nullptr, T, H, M->qd, st, M->d_err, M->tc_ws,
                               M->tc_ws_bytes));
       TIMED(Q2_K_NORM, launch_add_rms_norm(M->x, nullptr, M->h, w.post_norm, T, H, m.eps, dt, st, pdl));
       TIMED(Q2_K_GATE_UP, tc_gemm(M->s, I, Q2_BF16, TC_EPI_SWIGLU, M->h, w.wgu, nullptr, T, 2 * I, H, st,
-                                    M->tc_ws, M->tc_ws_bytes));
-      TIMED(Q2_K_DOWN, tc_gemm(M->x, H, Q2_BF16, TC_EPI_RESID, M->s, w.wd, nullptr, T, H, I, st, M->tc_ws,
+                                    M->d_err, M->tc_ws, M->tc_ws_bytes));
+      TIMED(Q2_K_DOWN, tc_gemm(M->x, H, Q2_BF16, TC_EPI_RESID, M->s, w.wd, nullptr, T, H, I, st, M->d_err, M->tc_ws,
                                  M->tc_ws_bytes));
       if (l + 1 < m.n_layers)
         TIMED(Q2_K_NORM, launch_add_rms_norm(M->x, nullptr, M->h, M->layers[l + 1].in_norm, T, H, m.eps,
@@ -350,10 +357,14 @@ q2_status run_head(q2_model* M, int r0, int rows, int lrow, cudaStream_t st, boo
 // ---- the fused bf16 decode path (batch <= kDecodeMaxBatch): five kernels
 // per layer, norms/RoPE/KV append/SwiGLU/residual adds in the linears'
 // prologues and epilogues, split attention with its combine folded in.
+bool use_stream(const q2_model* M, int B) {
+  // AUTO: the streaming step at batch 1.
+  return M->streaming && B == 1 && (M->path == Q2_PATH_STREAM || M->path == Q2_PATH_AUTO);
+}
 bool use_persistent(const q2_model* M, int B) {
   // AUTO: the persistent step where it is measured faster than the per-layer
-  // kernels (2 <= B <= 4 on B200; at B = 1 the per-layer kernels win).
-  return M->persistent && B >= 1 && B <= kPMaxBatch &&
+  // kernels (2 <= B <= 4 on B200).
+  return !use_stream(M, B) && M->persistent && B >= 1 && B <= kPMaxBatch &&
          (M->path == Q2_PATH_PERSISTENT || (M->path == Q2_PATH_AUTO && B >= 2));
 }
 bool use_fused(const q2_model* M, int B) {
@@ -411,6 +422,62 @@ q2_status persistent_step(q2_model* M, int B, bool head, bool embed_in, cudaStre
   if (trace)
     Q2_CUDA_TRY(cudaMemsetAsync(M->d_trace, 0, (5 * (size_t)m.n_layers + 1) * 4 * sizeof(unsigned long long), st));
   TIMED(Q2_K_STEP, launch_pdecode(p, M->kmap, M->vmap, st));
+  return Q2_OK;
+}
+
+// The batch-1 step (or the layers alone) as one streaming cooperative launch.
+q2_status stream_step(q2_model* M, bool head, bool embed_in, cudaStream_t st, bool trace = false,
+                      unsigned long long* ctrace = nullptr) {
+  const q2_meta& m = M->m;
+  SDecode p = {};
+  p.layers = M->d_layers;
+  p.L = m.n_layers;
+  p.H = m.hidden;
+  p.I = m.intermediate;
+  p.V = m.vocab;
+  p.nh = m.n_heads;
+  p.nkv = m.n_kv_heads;
+  p.hd = m.head_dim;
+  p.qkvd = M->qkvd;
+  p.qd = M->qd;
+  p.max_seq = m.max_seq;
+  p.Bmax = m.max_batch;
+  p.nsplit = decode_splits(M, 1);
+  p.eps = m.eps;
+  p.scale = 1.0f / sqrtf((float)m.head_dim);
+  p.embed_in = embed_in ? 1 : 0;
+  p.run_head = head ? 1 : 0;
+  p.embed = M->embed;
+  p.lm_head = M->lm_head;
+  p.final_norm = M->final_norm;
+  p.ids = M->d_ids;
+  p.x = M->x;
+  p.qb = M->qb;
+  p.att = M->att;
+  p.s = M->s;
+  p.kc = M->kc;
+  p.vc = M->vc;
+  p.kv_layer_stride = M->kv_layer_stride;
+  p.rope = M->rope;
+  p.lens = M->d_len;
+  p.part_o = (float*)M->attn_scratch;
+  p.part_ml = p.part_o + (size_t)m.n_heads * p.nsplit * m.head_dim;
+  p.logits = M->logits;
+  p.am_val = M->lm_val;
+  p.am_idx = M->lm_idx;
+  p.next = M->d_next;
+  p.sync = M->d_sync;
+  p.trace = trace ? M->d_trace : nullptr;
+  p.ctrace = ctrace;
+  p.err = M->d_err;
+  p.ring = M->sd_ring;
+  p.l2_ahead = M->sd_l2_ahead;
+  p.deadline_ns = M->wait_ns;
+  p.stall_phase = M->stall_phase;
+  Q2_CUDA_TRY(cudaMemsetAsync(M->d_sync, 0, sdecode_sync_words(m.n_layers, m.n_kv_heads) * sizeof(unsigned), st));
+  if (trace)
+    Q2_CUDA_TRY(cudaMemsetAsync(M->d_trace, 0, (5 * (size_t)m.n_layers + 1) * 4 * sizeof(unsigned long long), st));
+  TIMED(Q2_K_STEP, launch_sdecode(p, M->kmap, M->vmap, st));
   return Q2_OK;
 }
 
@@ -535,6 +602,7 @@ q2_status decode_body_fused(q2_model* M, int B, cudaStream_t st) {
 }
 
 q2_status decode_body(q2_model* M, int B, cudaStream_t st) {
+  if (use_stream(M, B)) return stream_step(M, true, true, st);
   if (use_persistent(M, B)) return persistent_step(M, B, true, true, st);
   if (use_fused(M, B)) return decode_body_fused(M, B, st);
   const bool pdl = true;
@@ -729,7 +797,8 @@ q2_status q2_model_create(const q2_meta* meta, int device, q2_model** out) {
   al.push_back({(void**)&M->d_counters, ((size_t)m.max_batch * m.n_kv_heads + 16) * sizeof(unsigned)});
   al.push_back({(void**)&M->lm_val, (size_t)num_sms() * kDecodeMaxBatch * sizeof(float)});
   al.push_back({(void**)&M->lm_idx, (size_t)num_sms() * kDecodeMaxBatch * sizeof(int64_t)});
-  al.push_back({(void**)&M->d_sync, pdecode_sync_words(m.n_layers) * sizeof(unsigned)});
+  const size_t sync_words = std::max(pdecode_sync_words(m.n_layers), sdecode_sync_words(m.n_layers, m.n_kv_heads));
+  al.push_back({(void**)&M->d_sync, sync_words * sizeof(unsigned)});
   al.push_back({(void**)&M->d_layers, (size_t)m.n_layers * sizeof(PLayer)});
   al.push_back({(void**)&M->d_trace, (5 * (size_t)m.n_layers + 1) * 4 * sizeof(unsigned long long)});
   if (M->dt == Q2_BF16) {
@@ -787,9 +856,21 @@ q2_status q2_model_create(const q2_meta* meta, int device, q2_model** out) {
     M->fused = (vs == Q2_OK) && rows < (1ull << 31);
     M->persistent = M->fused && pdecode_supported(m.hidden, m.intermediate, m.vocab, m.n_heads,
                                                   m.n_kv_heads, m.head_dim, M->qkvd, M->qd);
+    M->streaming = M->fused && sdecode_supported(m.hidden, m.intermediate, m.vocab, m.n_heads,
+                                                 m.n_kv_heads, m.head_dim, M->qkvd, M->qd);
+    M->sd_ring = sdecode_default_ring();
+    // Tuning knobs of the persistent and streaming steps (for measurements).
     if (const char* env = getenv("Q2_PDECODE_L2_AHEAD")) {
       const int v = atoi(env);
       if (v >= 0 && v <= 256) M->l2_ahead = v;
+    }
+    if (const char* env = getenv("Q2_SDECODE_RING")) {
+      const int v = atoi(env);
+      if (v >= 2 && v <= 16) M->sd_ring = v;
+    }
+    if (const char* env = getenv("Q2_SDECODE_L2_AHEAD")) {
+      const int v = atoi(env);
+      if (v >= 0 && v <= 256) M->sd_l2_ahead = v;
     }
     clear_error();
   }
@@ -953,8 +1034,11 @@ q2_status q2_model_forward_hidden(q2_model* M, const void* x_in, int B, void* x_
   Q2_TRY(check_stream_device(M, st));
   const size_t bytes = (size_t)B * M->m.hidden * M->es;
   Q2_CUDA_TRY(cudaMemcpyAsync(M->x, x_in, bytes, cudaMemcpyDeviceToDevice, st));
-  if (use_persistent(M, B)) {
-    Q2_TRY(persistent_step(M, B, false, false, st));  // advances the lengths itself
+  if (use_stream(M, B) || use_persistent(M, B)) {
+    if (use_stream(M, B))
+      Q2_TRY(stream_step(M, false, false, st));  // advances the length itself
+    else
+      Q2_TRY(persistent_step(M, B, false, false, st));  // advances the lengths itself
     Q2_CUDA_TRY(cudaMemcpyAsync(x_out, M->x, bytes, cudaMemcpyDeviceToDevice, st));
     for (int b = 0; b < B; ++b) M->h_len[b] += 1;
     return Q2_OK;
@@ -1066,9 +1150,67 @@ q2_status q2_model_check_error(q2_model* M, void* stream) {
   if (v) {
     int zero = 0;
     Q2_CUDA_TRY(cudaMemcpy(M->d_err, &zero, sizeof zero, cudaMemcpyHostToDevice));
-    set_error("a model kernel saw a token id outside [0, vocab)");
-    return Q2_ERR_INDEX;
+    return device_error_status(v, "model_check_error");
   }
+  return Q2_OK;
+}
+
+q2_status q2_test_model_raise_error(q2_model* M, int bits, void* stream) {
+  clear_error();
+  Q2_CHECK_ARG(M, Q2_ERR_INVALID_ARG, "test_model_raise_error: NULL model");
+  Q2_CHECK_ARG(bits > 0 && bits <= (kErrIndex | kErrTimeout), Q2_ERR_INVALID_ARG,
+               "test_model_raise_error: bits must be 1, 2 or 3");
+  DeviceGuard g(M->device);
+  cudaStream_t st = as_stream(stream);
+  int cur = 0;
+  Q2_CUDA_TRY(cudaMemcpyAsync(&cur, M->d_err, sizeof cur, cudaMemcpyDeviceToHost, st));
+  Q2_CUDA_TRY(cudaStreamSynchronize(st));
+  cur |= bits;
+  Q2_CUDA_TRY(cudaMemcpyAsync(M->d_err, &cur, sizeof cur, cudaMemcpyHostToDevice, st));
+  Q2_CUDA_TRY(cudaStreamSynchronize(st));
+  return Q2_OK;
+}
+
+q2_status q2_test_trace_stream_step(q2_model* M, const int64_t* ids, unsigned long long* out, size_t n,
+                                    int* grid, void* stream) {
+  clear_error();
+  Q2_CHECK_ARG(M && ids && out && grid, Q2_ERR_INVALID_ARG, "trace_stream_step: NULL argument");
+  Q2_CHECK_ARG(M->streaming, Q2_ERR_STATE, "trace_stream_step: the streaming step does not support this model");
+  Q2_CHECK_ARG(M->h_len[0] < M->m.max_seq, Q2_ERR_CAPACITY, "trace_stream_step: the sequence is full");
+  const size_t words = (5 * (size_t)M->m.n_layers + 1) * num_sms() * 4;
+  Q2_CHECK_ARG(n >= words, Q2_ERR_SHAPE, "trace_stream_step: output too small");
+  DeviceGuard g(M->device);
+  cudaStream_t st = as_stream(stream);
+  Q2_TRY(check_stream_device(M, st));
+  unsigned long long* d = nullptr;
+  Q2_CUDA_TRY(cudaMalloc(&d, words * sizeof(unsigned long long)));
+  Q2_CUDA_TRY(cudaMemsetAsync(d, 0, words * sizeof(unsigned long long), st));
+  const int saved = M->h_len[0];
+  Q2_CUDA_TRY(cudaMemcpyAsync(M->d_ids, ids, sizeof(int64_t), cudaMemcpyDeviceToDevice, st));
+  q2_status s = stream_step(M, true, true, st, false, d);
+  if (s == Q2_OK) s = cudaMemcpyAsync(out, d, words * sizeof(unsigned long long), cudaMemcpyDeviceToHost, st) == cudaSuccess ? Q2_OK : Q2_ERR_CUDA;
+  if (s == Q2_OK) s = cudaStreamSynchronize(st) == cudaSuccess ? Q2_OK : Q2_ERR_CUDA;
+  cudaFree(d);
+  // the traced step leaves the model where it was
+  if (s == Q2_OK) s = cudaMemcpy(M->d_len, &saved, sizeof(int), cudaMemcpyHostToDevice) == cudaSuccess ? Q2_OK : Q2_ERR_CUDA;
+  *grid = num_sms();
+  if (s != Q2_OK && q2_last_error()[0] == 0) set_error("trace_stream_step: a CUDA call failed");
+  return s;
+}
+
+q2_status q2_test_set_wait_fault(q2_model* M, int phase, unsigned long long deadline_ns) {
+  clear_error();
+  Q2_CHECK_ARG(M, Q2_ERR_INVALID_ARG, "test_set_wait_fault: NULL model");
+  Q2_CHECK_ARG(phase >= -1 && phase <= 5 * M->m.n_layers, Q2_ERR_INVALID_ARG,
+               "test_set_wait_fault: phase outside [-1, 5 * n_layers]");
+  Q2_CHECK_ARG(deadline_ns >= 1000, Q2_ERR_INVALID_ARG, "test_set_wait_fault: deadline below 1 us");
+  DeviceGuard g(M->device);
+  cudaDeviceSynchronize();
+  // captured steps hold the old settings: drop them
+  for (auto& kv : M->graphs) cudaGraphExecDestroy(kv.second);
+  M->graphs.clear();
+  M->stall_phase = phase;
+  M->wait_ns = phase < 0 ? 200ull * 1000 * 1000 : deadline_ns;
   return Q2_OK;
 }
 
@@ -1092,7 +1234,7 @@ q2_status q2_model_time_kernels(q2_model* M, const int64_t* ids, int B, int step
   DeviceGuard g(M->device);
   cudaStream_t st = as_stream(stream);
   Q2_TRY(check_stream_device(M, st));
-  if (use_persistent(M, B)) {
+  if (use_stream(M, B) || use_persistent(M, B)) {
     // One kernel per step: per-phase critical-path times from the kernel's
     // own global-timer stamps (latest end of a phase minus the latest end of
     // the phase before), and the whole launch by CUDA events.
@@ -1108,7 +1250,10 @@ q2_status q2_model_time_kernels(q2_model* M, const int64_t* ids, int B, int step
     for (int r = 0; r < steps; ++r) {
       Q2_CUDA_TRY(cudaMemcpyAsync(M->d_ids, ids, B * sizeof(int64_t), cudaMemcpyDeviceToDevice, st));
       Q2_CUDA_TRY(cudaEventRecord(e0, st));
-      Q2_TRY(persistent_step(M, B, true, true, st, true));
+      if (use_stream(M, B))
+        Q2_TRY(stream_step(M, true, true, st, true));
+      else
+        Q2_TRY(persistent_step(M, B, true, true, st, true));
       Q2_CUDA_TRY(cudaEventRecord(e1, st));
       Q2_CUDA_TRY(cudaStreamSynchronize(st));
       float ms = 0.f;
@@ -1235,8 +1380,10 @@ q2_status q2_model_head(q2_model* M, const void* x, int rows, int64_t* next, flo
 q2_status q2_model_set_decode_path(q2_model* M, int path) {
   clear_error();
   Q2_CHECK_ARG(M, Q2_ERR_INVALID_ARG, "set_decode_path: NULL model");
-  Q2_CHECK_ARG(path >= Q2_PATH_AUTO && path <= Q2_PATH_GENERIC, Q2_ERR_INVALID_ARG,
+  Q2_CHECK_ARG(path >= Q2_PATH_AUTO && path <= Q2_PATH_STREAM, Q2_ERR_INVALID_ARG,
                "set_decode_path: bad path");
+  Q2_CHECK_ARG(path != Q2_PATH_STREAM || M->streaming, Q2_ERR_STATE,
+               "set_decode_path: the streaming step does not support this model");
   Q2_CHECK_ARG(path != Q2_PATH_PERSISTENT || M->persistent, Q2_ERR_STATE,
                "set_decode_path: the persistent kernel does not support this model");
   Q2_CHECK_ARG(path != Q2_PATH_KERNELS || M->fused, Q2_ERR_STATE,

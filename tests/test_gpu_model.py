@@ -276,6 +276,73 @@ def test_capacity_and_index_errors(tiny_w):
     assert e.value.status == "Q2_ERR_CAPACITY"
 
 
+def test_error_words_map_bits_to_statuses(tiny_w):
+    """Each bit of a device error word has its own status: 1 (a token id
+    outside the vocabulary) -> Q2_ERR_INDEX, 2 (a bounded wait ran out) ->
+    Q2_ERR_TIMEOUT, which takes precedence; reading clears the word."""
+    shape = TINY["shape"]
+    gm = q2.Model(shape, max_seq=8)
+    gm.load(tiny_w)
+    for bits, status in ((1, "Q2_ERR_INDEX"), (2, "Q2_ERR_TIMEOUT"), (3, "Q2_ERR_TIMEOUT")):
+        gm.test_raise_error(bits)
+        with pytest.raises(q2.Q2Error) as e:
+            gm.check_error()
+        assert e.value.status == status
+        if bits == 3:
+            assert "token id" in str(e.value)
+        gm.check_error()  # cleared
+        q2.q2_test_raise_device_error(bits)
+        with pytest.raises(q2.Q2Error) as e:
+            q2.q2_check_device_error()
+        assert e.value.status == status
+        q2.q2_check_device_error()
+
+
+def test_stream_step_wait_that_runs_out_is_reported_and_recoverable(mid):
+    """A grid-phase counter of the streaming step that never completes (test
+    hook: one arrival more than the grid makes): every wait on it gives up at
+    its deadline, the step returns promptly, q2_model_check_error reports
+    Q2_ERR_TIMEOUT, and after the hook is cleared the model decodes exactly as
+    before."""
+    import time
+
+    shape, w = mid
+    gm = q2.Model(shape, max_seq=64)
+    gm.load(w)
+    gm.set_decode_path("stream")
+    prompt = synth.prompt_ids(shape, 12, 8).cuda()
+
+    def run(n):
+        gm.reset_kv()
+        nxt = gm.prefill(prompt, [12])
+        out = []
+        for _ in range(n):
+            nxt, lg = gm.decode_step(nxt, want_logits=True)
+            out.append(lg.clone())
+        return nxt, out
+
+    _, ref = run(3)
+    gm.check_error()
+    gm.reset_kv()
+    nxt = gm.prefill(prompt, [12])
+    gm.test_set_wait_fault(5 * 1 + 2, 2_000_000)  # layer 1's o phase; 2 ms deadline
+    gm.set_graphs(False)  # an eager launch: the time is the step's own
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    gm.decode_step(nxt)
+    torch.cuda.synchronize()
+    dt = time.perf_counter() - t0
+    gm.set_graphs(True)
+    with pytest.raises(q2.Q2Error) as e:
+        gm.check_error()
+    assert e.value.status == "Q2_ERR_TIMEOUT"
+    assert dt < 0.15, dt  # one 2 ms deadline, not one per phase (nor the 200 ms default)
+    gm.test_set_wait_fault(-1)
+    _, again = run(3)
+    gm.check_error()
+    assert all(bits_equal(a, b) for a, b in zip(ref, again))
+
+
 def test_decode_step_host_matches_device_path(tiny_w):
     shape = TINY["shape"]
     prompt = synth.prompt_ids(shape, 10, 3)
@@ -302,8 +369,9 @@ def test_decode_step_host_matches_device_path(tiny_w):
 
 @pytest.mark.parametrize("B", [1, 3])
 def test_decode_paths_agree_with_each_other_and_the_oracle(mid, B):
-    """The persistent step, the five-kernel fused path and the per-operator
-    path compute the same decode steps (teacher-forced ids, B sequences)."""
+    """The streaming step (batch 1), the persistent step, the five-kernel fused
+    path and the per-operator path compute the same decode steps
+    (teacher-forced ids, B sequences)."""
     shape, w = mid
     lens = [20, 33, 7][:B]
     prompts = [synth.prompt_ids(shape, n, 40 + b, seq=b) for b, n in enumerate(lens)]
@@ -311,7 +379,8 @@ def test_decode_paths_agree_with_each_other_and_the_oracle(mid, B):
     gm = q2.Model(shape, max_seq=128, max_batch=4)
     gm.load(w)
     out = {}
-    for path in ("persistent", "kernels", "generic"):
+    paths = ("stream", "persistent", "kernels", "generic") if B == 1 else ("persistent", "kernels", "generic")
+    for path in paths:
         gm.set_decode_path(path)
         gm.reset_kv()
         gm.prefill(torch.cat(prompts).cuda(), lens)
@@ -321,7 +390,7 @@ def test_decode_paths_agree_with_each_other_and_the_oracle(mid, B):
             lg.append(l.cpu())
         gm.check_error()
         out[path] = lg
-    for path in ("persistent", "kernels"):
+    for path in paths[:-1]:
         for a, b in zip(out[path], out["generic"]):
             for r in range(B):
                 assert_bf16_logits(a[r], b[r], f"{path} vs generic, row {r}")
@@ -330,7 +399,8 @@ def test_decode_paths_agree_with_each_other_and_the_oracle(mid, B):
     om.load({k: t.cpu() for k, t in w.items()})
     om.forward(0, prompts[0])
     _, ref = om.forward(0, feeds[0][:1])
-    assert_bf16_logits(out["persistent"][0][0], ref, "persistent vs oracle")
+    for path in paths[:2]:
+        assert_bf16_logits(out[path][0][0], ref, f"{path} vs oracle")
 
 
 def test_persistent_step_is_deterministic_and_graph_safe(mid):
@@ -353,3 +423,36 @@ def test_persistent_step_is_deterministic_and_graph_safe(mid):
     for x, y, z in zip(*runs):
         assert bits_equal(x, y) and bits_equal(x, z)
     assert gm.get_seq_len(0) == gm.get_seq_len(1) == 18
+
+
+def test_stream_step_is_deterministic_and_graph_safe(mid):
+    """The batch-1 streaming step: graphs and eager launches, reruns after
+    reset_kv, all bit-identical (fixed summation orders everywhere); the
+    length advances once per step."""
+    shape, w = mid
+    gm = q2.Model(shape, max_seq=300, max_batch=1)
+    gm.load(w)
+    gm.set_decode_path("stream")
+    prompt = synth.prompt_ids(shape, 150, 9).cuda()
+    runs = []
+    for graphs in (True, False, True):
+        gm.reset_kv()
+        gm.set_graphs(graphs)
+        nxt = gm.prefill(prompt, [150])
+        lgs, toks = [], []
+        for _ in range(6):
+            nxt, lg = gm.decode_step(nxt, want_logits=True)
+            lgs.append(lg.clone())
+            toks.append(int(nxt[0]))
+        runs.append((lgs, toks))
+        gm.check_error()
+    for (x, tx), (y, ty) in zip(runs, runs[1:]):
+        assert tx == ty
+        assert all(bits_equal(a, b) for a, b in zip(x, y))
+    assert gm.get_seq_len(0) == 156
+    # the token is the argmax of the step's own logits (lowest index on ties)
+    assert toks_match_argmax(runs[0][0], runs[0][1])
+
+
+def toks_match_argmax(logits, toks):
+    return all(int(torch.argmax(l[0]).item()) == t for l, t in zip(logits, toks))
