@@ -91,6 +91,8 @@ struct q2_model {
   int sd_ring = 0;                 // streaming step: weight ring slots (Q2_SDECODE_RING overrides)
   int sd_l2_ahead = 0;             // streaming step: slots pulled into L2 ahead of the ring
   unsigned long long wait_ns = 200ull * 1000 * 1000;  // bound of every device-side wait
+  uint64_t* sd_ll = nullptr;       // streaming step: tagged exchange words
+  unsigned* sd_epoch = nullptr;    // streaming step: step counter (never reset)
   int stall_phase = -1;            // test hook: a phase counter that never completes
   int path = Q2_PATH_AUTO;
   // Weight stages each CTA of the persistent step pulls into L2 ahead of its
@@ -452,19 +454,14 @@ q2_status stream_step(q2_model* M, bool head, bool embed_in, cudaStream_t st, bo
   p.final_norm = M->final_norm;
   p.ids = M->d_ids;
   p.x = M->x;
-  p.qb = M->qb;
-  p.att = M->att;
-  p.s = M->s;
   p.kc = M->kc;
   p.vc = M->vc;
   p.kv_layer_stride = M->kv_layer_stride;
   p.rope = M->rope;
   p.lens = M->d_len;
-  p.part_o = (float*)M->attn_scratch;
-  p.part_ml = p.part_o + (size_t)m.n_heads * p.nsplit * m.head_dim;
+  p.ll = sdecode_ll_carve(M->sd_ll, m.hidden, m.intermediate, m.n_heads, m.n_kv_heads, m.head_dim, num_sms());
+  p.epoch = M->sd_epoch;
   p.logits = M->logits;
-  p.am_val = M->lm_val;
-  p.am_idx = M->lm_idx;
   p.next = M->d_next;
   p.sync = M->d_sync;
   p.trace = trace ? M->d_trace : nullptr;
@@ -474,7 +471,7 @@ q2_status stream_step(q2_model* M, bool head, bool embed_in, cudaStream_t st, bo
   p.l2_ahead = M->sd_l2_ahead;
   p.deadline_ns = M->wait_ns;
   p.stall_phase = M->stall_phase;
-  Q2_CUDA_TRY(cudaMemsetAsync(M->d_sync, 0, sdecode_sync_words(m.n_layers, m.n_kv_heads) * sizeof(unsigned), st));
+  Q2_CUDA_TRY(cudaMemsetAsync(M->d_sync, 0, sdecode_sync_words() * sizeof(unsigned), st));
   if (trace)
     Q2_CUDA_TRY(cudaMemsetAsync(M->d_trace, 0, (5 * (size_t)m.n_layers + 1) * 4 * sizeof(unsigned long long), st));
   TIMED(Q2_K_STEP, launch_sdecode(p, M->kmap, M->vmap, st));
@@ -797,8 +794,13 @@ q2_status q2_model_create(const q2_meta* meta, int device, q2_model** out) {
   al.push_back({(void**)&M->d_counters, ((size_t)m.max_batch * m.n_kv_heads + 16) * sizeof(unsigned)});
   al.push_back({(void**)&M->lm_val, (size_t)num_sms() * kDecodeMaxBatch * sizeof(float)});
   al.push_back({(void**)&M->lm_idx, (size_t)num_sms() * kDecodeMaxBatch * sizeof(int64_t)});
-  const size_t sync_words = std::max(pdecode_sync_words(m.n_layers), sdecode_sync_words(m.n_layers, m.n_kv_heads));
+  const size_t sync_words = std::max(pdecode_sync_words(m.n_layers), sdecode_sync_words());
   al.push_back({(void**)&M->d_sync, sync_words * sizeof(unsigned)});
+  if (M->dt == Q2_BF16 && m.head_dim % 2 == 0 && m.n_heads % m.n_kv_heads == 0) {
+    al.push_back({(void**)&M->sd_ll, sdecode_ll_words(m.hidden, m.intermediate, m.n_heads, m.n_kv_heads,
+                                                      m.head_dim, num_sms()) * sizeof(uint64_t)});
+    al.push_back({(void**)&M->sd_epoch, sizeof(unsigned)});
+  }
   al.push_back({(void**)&M->d_layers, (size_t)m.n_layers * sizeof(PLayer)});
   al.push_back({(void**)&M->d_trace, (5 * (size_t)m.n_layers + 1) * 4 * sizeof(unsigned long long)});
   if (M->dt == Q2_BF16) {
@@ -858,7 +860,8 @@ q2_status q2_model_create(const q2_meta* meta, int device, q2_model** out) {
                                                   m.n_kv_heads, m.head_dim, M->qkvd, M->qd);
     M->streaming = M->fused && sdecode_supported(m.hidden, m.intermediate, m.vocab, m.n_heads,
                                                  m.n_kv_heads, m.head_dim, M->qkvd, M->qd);
-    M->sd_ring = sdecode_default_ring();
+    M->sd_ring = std::min(6, sdecode_max_ring(m.n_layers));
+    M->streaming = M->streaming && M->sd_ring >= 2 && M->sd_ll != nullptr;
     // Tuning knobs of the persistent and streaming steps (for measurements).
     if (const char* env = getenv("Q2_PDECODE_L2_AHEAD")) {
       const int v = atoi(env);

@@ -22,27 +22,25 @@ constexpr int kThreads = kCT + 32;     // + the producer warp
 constexpr int kSB = 24576;             // weight ring slot: 8 rows of K = 1536, or one down row
 constexpr int kAT = 64;                // attention keys per tile
 constexpr int kHD = 128;               // head dim of this kernel
+constexpr int kHalf = kHD / 2;
 constexpr int kTile = kAT * kHD * 2;   // one K (or V) tile
 constexpr int kAGMax = 8;              // query heads per kv head
 constexpr int kYMax = 256;             // rows per CTA of a short-row phase (parked row results)
 constexpr int kDMax = 64;              // rows per CTA of the o and down phases
 constexpr int kQMax = 64;              // q/k/v rows per CTA (staged epilogue operands)
-constexpr int kSplitMax = 64;
-constexpr int kLMax = 128;             // layers (the layer table sits in shared memory)
+constexpr int kHMax = 2048;            // hidden size (the staged input vector)
+constexpr int kSplitMax = kSDecodeSplitMax;
 constexpr size_t kSmemMax = 232448;    // 227 KB per CTA
 constexpr float kLog2e = 1.4426950408889634f;
 
 enum { PH_QKV = 0, PH_ATTN = 1, PH_O = 2, PH_GU = 3, PH_DOWN = 4, PH_HEAD = 5 };
-
-// s_flags slots
-enum { F_LAST = 0, F_MERGE = 1, F_PRE = 2, F_STALE = 3, F_LEN = 4 };
 
 __host__ __device__ inline size_t up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Shared-memory map (offsets from a 1024-byte aligned base: the attention
 // tiles are 128-byte-swizzled TMA boxes).
 struct SLay {
-  size_t tiles, ring, layers, wts, mraw, yrow, part, xres, ebias, ecs, mlw, amv, ami, bars, flags, total;
+  size_t tiles, ring, layers, yrow, part, xres, ebias, ecs, mlw, amv, ami, xbuf, qst, kvn, bars, flags, total;
 };
 
 __host__ __device__ inline SLay slayout(int ring, int L) {
@@ -54,10 +52,6 @@ __host__ __device__ inline SLay slayout(int ring, int L) {
   o += (size_t)ring * kSB;
   Y.layers = o;  // [L] layer weight pointers
   o = up(o + (size_t)L * sizeof(PLayer), 16);
-  Y.wts = o;  // [kAGMax][kSplitMax] split weights of the merge
-  o += (size_t)kAGMax * kSplitMax * 4;
-  Y.mraw = o;  // [kAGMax][kSplitMax] split maxima of the merge
-  o += (size_t)kAGMax * kSplitMax * 4;
   Y.yrow = o;  // [kYMax] row results of a short-row phase
   o += (size_t)kYMax * 4;
   Y.part = o;  // [kCW][kDMax] per-warp column-slice sums of the down rows
@@ -74,6 +68,12 @@ __host__ __device__ inline SLay slayout(int ring, int L) {
   o += kCW * 4;
   Y.ami = up(o, 8);  // [kCW] per-warp argmax indices
   o = Y.ami + kCW * 8;
+  Y.xbuf = up(o, 16);  // [kHMax] bf16: the phase's input vector
+  o = Y.xbuf + (size_t)kHMax * 2;
+  Y.qst = o;  // [kAGMax][kHD] bf16: one kv head's query heads
+  o += (size_t)kAGMax * kHD * 2;
+  Y.kvn = o;  // [2][kHD] bf16: the new K and V rows of that kv head
+  o += 2 * (size_t)kHD * 2;
   Y.bars = up(o, 8);  // full[ring], empty[ring], abar[2]
   o = Y.bars + (2 * (size_t)ring + 2) * 8;
   Y.flags = o;
@@ -88,20 +88,8 @@ __device__ __forceinline__ uint64_t gtimer() {
   return t;
 }
 
-__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
-  unsigned v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
-__device__ __forceinline__ unsigned atom_add_release(unsigned* p, unsigned v) {
-  unsigned old;
-  asm volatile("atom.add.release.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-  return old;
-}
-
-__device__ __forceinline__ void fence_proxy_async_global() {
-  asm volatile("fence.proxy.async.global;" ::: "memory");
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 // Orders this thread's generic-proxy writes to shared memory before later
@@ -110,39 +98,101 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
-
 // Consumer-warps-only barrier (the producer warp never joins it).
 __device__ __forceinline__ void csync() { asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory"); }
 
-// mbarrier wait bounded by a deadline on the global timer; false if it ran out.
-__device__ __forceinline__ bool bwait(uint64_t* bar, uint32_t parity, uint64_t deadline_ns) {
+// mbarrier wait bounded by a deadline on the global timer; false if it ran
+// out.  With `gave_up` given, it also stops as soon as some wait of the launch
+// has given up (the step's results are undefined by then).
+__device__ __forceinline__ bool bwait(uint64_t* bar, uint32_t parity, uint64_t deadline_ns,
+                                      const unsigned* gave_up = nullptr) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = gtimer();
   for (;;) {
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(bar, parity)) return true;
     if (gtimer() - t0 > deadline_ns) return false;
+    if (gave_up && *reinterpret_cast<const volatile unsigned*>(gave_up) != 0u) return false;
   }
 }
 
-// Wait until a grid counter reaches `target`, bounded by the deadline; once
-// some wait of this launch has run out (`gave_up` set) it gives up at once,
-// so a stalled step ends after one deadline rather than one per phase.
-__device__ __forceinline__ bool gwait(const unsigned* ctr, unsigned target, uint64_t deadline_ns,
-                                      const unsigned* gave_up) {
-  if (ld_acquire(ctr) >= target) return true;
-  const uint64_t t0 = gtimer();
-  for (unsigned it = 1;; ++it) {
-    if (ld_acquire(ctr) >= target) return true;
-    if ((it & 63u) == 0) {
-      if (*reinterpret_cast<const volatile unsigned*>(gave_up)) return false;
-      if (gtimer() - t0 > deadline_ns) return false;
+// ---------------------------------------------------------- tagged words
+// A word is {u32 data, u32 tag}; 8-byte accesses are single-copy atomic, so a
+// reader sees data and tag of the same store.  Stores and loads are volatile
+// (no L1 caching): they meet in L2.
+__device__ __forceinline__ void ll_put(uint64_t* w, uint32_t data, uint32_t tag) {
+  const uint64_t v = ((uint64_t)tag << 32) | data;
+  asm volatile("st.volatile.global.u64 [%0], %1;" ::"l"(w), "l"(v) : "memory");
+}
+// Two consecutive words (16-byte aligned) in one vector store.
+__device__ __forceinline__ void ll_put2(uint64_t* w, uint32_t d0, uint32_t d1, uint32_t tag) {
+  asm volatile("st.volatile.global.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(w), "r"(d0), "r"(tag), "r"(d1),
+               "r"(tag)
+               : "memory");
+}
+
+// Bounded polling of tagged words.  Once any wait of the launch has run out
+// (`gave_up`), a poll that does not succeed at once gives up too, so a
+// stalled step ends after one deadline rather than one per wait.
+struct Poll {
+  uint64_t deadline_ns;
+  unsigned* gave_up;
+  int* err;
+  __device__ void fail() const {
+    atomicOr(err, 2);
+    atomicExch(gave_up, 1u);
+  }
+  __device__ bool stop(uint64_t t0) const {
+    return *reinterpret_cast<volatile unsigned*>(gave_up) != 0u || gtimer() - t0 > deadline_ns;
+  }
+  // one word
+  __device__ uint32_t get(const uint64_t* w, uint32_t tag) const {
+    uint64_t v;
+    asm volatile("ld.volatile.global.u64 %0, [%1];" : "=l"(v) : "l"(w) : "memory");
+    if ((uint32_t)(v >> 32) == tag) return (uint32_t)v;
+    const uint64_t t0 = gtimer();
+    for (unsigned it = 1;; ++it) {
+      asm volatile("ld.volatile.global.u64 %0, [%1];" : "=l"(v) : "l"(w) : "memory");
+      if ((uint32_t)(v >> 32) == tag) return (uint32_t)v;
+      if ((it & 15u) == 0 && stop(t0)) {
+        fail();
+        return (uint32_t)v;
+      }
     }
   }
+  // two consecutive words (16-byte aligned)
+  __device__ uint2 get2(const uint64_t* w, uint32_t tag) const {
+    uint32_t d0, t0_, d1, t1_;
+    asm volatile("ld.volatile.global.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(d0), "=r"(t0_), "=r"(d1), "=r"(t1_)
+                 : "l"(w)
+                 : "memory");
+    if (t0_ == tag && t1_ == tag) return make_uint2(d0, d1);
+    const uint64_t t0 = gtimer();
+    for (unsigned it = 1;; ++it) {
+      asm volatile("ld.volatile.global.v4.u32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(d0), "=r"(t0_), "=r"(d1), "=r"(t1_)
+                   : "l"(w)
+                   : "memory");
+      if (t0_ == tag && t1_ == tag) return make_uint2(d0, d1);
+      if ((it & 15u) == 0 && stop(t0)) {
+        fail();
+        return make_uint2(d0, d1);
+      }
+    }
+  }
+};
+
+__device__ __forceinline__ uint32_t bf2_bits(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
 }
+__device__ __forceinline__ uint32_t bf2_bits(bf16 lo, bf16 hi) {
+  return (uint32_t)*reinterpret_cast<const uint16_t*>(&lo) |
+         ((uint32_t)*reinterpret_cast<const uint16_t*>(&hi) << 16);
+}
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
 __device__ __forceinline__ float silu_mul(float gv, float uv) { return uv * (gv / (1.0f + expf(-gv))); }
 
@@ -176,18 +226,14 @@ __device__ __forceinline__ void mma16816(float* c, uint32_t a0, uint32_t a2, uin
       : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&v);
-}
-
 __device__ __forceinline__ int phase_kind(int L, int ph) { return ph == 5 * L ? PH_HEAD : ph % 5; }
 
 // The weight rows a CTA streams in one phase: rows [r0, r1) of w [N][K], in
-// stages of rs whole rows.  Rows are dealt out in contiguous blocks, in units
-// of row pairs where the epilogue needs both members of a pair (RoPE
-// partners, gate/up).  The o and down phases split their rows alike, so a CTA
-// owns the same rows of the residual stream in both.
+// stages of rs whole rows.  Rows are dealt out in contiguous blocks of whole
+// units: a RoPE pair for q/k/v (one tagged word of q, k or v), two rows for o
+// and down (one word of x), two gate/up pairs for gate/up (one word of s).
+// The o and down phases split their rows alike, so a CTA owns the same rows
+// of the residual stream in both.
 struct PW {
   const bf16* w;
   int K, r0, r1, rs;
@@ -201,9 +247,9 @@ __device__ __forceinline__ bool phase_w(const SDecode& p, const PLayer* layers, 
   int N, unit;
   switch (kind) {
     case PH_QKV: o.w = (const bf16*)lw->wqkv; N = p.qkvd; o.K = p.H; unit = 2; break;
-    case PH_O: o.w = (const bf16*)lw->wo; N = p.H; o.K = p.qd; unit = 1; break;
-    case PH_GU: o.w = (const bf16*)lw->wgu; N = 2 * p.I; o.K = p.H; unit = 2; break;
-    case PH_DOWN: o.w = (const bf16*)lw->wd; N = p.H; o.K = p.I; unit = 1; break;
+    case PH_O: o.w = (const bf16*)lw->wo; N = p.H; o.K = p.qd; unit = 2; break;
+    case PH_GU: o.w = (const bf16*)lw->wgu; N = 2 * p.I; o.K = p.H; unit = 4; break;
+    case PH_DOWN: o.w = (const bf16*)lw->wd; N = p.H; o.K = p.I; unit = 2; break;
     default: o.w = (const bf16*)p.lm_head; N = p.V; o.K = p.H; unit = 1; break;
   }
   const long long units = N / unit;
@@ -258,8 +304,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* tiles = smem + Y.tiles;
   uint8_t* ring = smem + Y.ring;
   PLayer* layers = reinterpret_cast<PLayer*>(smem + Y.layers);
-  float* wts = reinterpret_cast<float*>(smem + Y.wts);
-  float* mraw = reinterpret_cast<float*>(smem + Y.mraw);
   float* yrow = reinterpret_cast<float*>(smem + Y.yrow);
   float* part = reinterpret_cast<float*>(smem + Y.part);
   float* xres = reinterpret_cast<float*>(smem + Y.xres);
@@ -268,17 +312,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* mlw = reinterpret_cast<float*>(smem + Y.mlw);
   float* amv = reinterpret_cast<float*>(smem + Y.amv);
   long long* ami = reinterpret_cast<long long*>(smem + Y.ami);
+  bf16* xbuf = reinterpret_cast<bf16*>(smem + Y.xbuf);
+  bf16* qst = reinterpret_cast<bf16*>(smem + Y.qst);
+  bf16* kvn = reinterpret_cast<bf16*>(smem + Y.kvn);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Y.bars);
   uint64_t* empty = full + RING;
   uint64_t* abar = empty + RING;
-  int* s_flags = reinterpret_cast<int*>(smem + Y.flags);
+  int* s_flags = reinterpret_cast<int*>(smem + Y.flags);  // [0] position, [1] step, [2] tiles pre-issued
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x, bid = blockIdx.x;
   const int nph = p.run_head ? 5 * L + 1 : 5 * L;
   const uint64_t dl = p.deadline_ns;
 
-  // the layer table in shared memory; the step's position
+  // the layer table in shared memory; the step's position and counter
   for (int i = tid; i < L * (int)(sizeof(PLayer) / 8); i += kThreads)
     reinterpret_cast<unsigned long long*>(layers)[i] = reinterpret_cast<const unsigned long long*>(p.layers)[i];
   if (tid == 0) {
@@ -289,13 +336,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&abar[0], 1);
     mbar_init(&abar[1], 1);
     fence_mbar_init();
-    s_flags[F_LEN] = __ldcg(p.lens);
-    s_flags[F_PRE] = 0;
-    s_flags[F_STALE] = -1;
+    s_flags[0] = __ldcg(p.lens);
+    s_flags[1] = (int)__ldcg(p.epoch);
+    s_flags[2] = 0;
   }
   __syncthreads();
-  const int pos = s_flags[F_LEN];  // the new token's position
-  const int alen = pos + 1;        // keys attended (the new token included)
+  const int pos = s_flags[0];  // the new token's position
+  const int alen = pos + 1;    // keys attended (the new token included)
+  // tag of phase ph's outputs in this step (unique per step and phase)
+  const uint32_t tbase = (uint32_t)s_flags[1] * (uint32_t)(nph + 1) + 1u;
+  auto wtag = [&](int ph) { return tbase + (uint32_t)ph; };
+  // what a reader of phase ph's outputs waits for (the test hook makes one phase's
+  // outputs unrecognisable to its readers)
+  auto rtag = [&](int ph) { return wtag(ph) ^ (ph == p.stall_phase ? 0x80000000u : 0u); };
 
   // ================================================================ producer
   // One lane walks this CTA's stages of the whole step and issues one bulk
@@ -313,8 +366,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       int slot = 0;
       uint32_t par = 0;
-      for (long long gs = 0; cur.valid(nph); ++gs) {
-        if (gs >= RING && !bwait(&empty[slot], par ^ 1u, dl)) atomicOr(p.err, 2);
+      long long gs = 0;
+      for (; cur.valid(nph); ++gs) {
+        if (gs >= RING && !bwait(&empty[slot], par ^ 1u, dl, p.sync)) {
+          // the consumers stopped: issuing into a slot still in use would
+          // break the ring's protocol, so stop here
+          atomicOr(p.err, 2);
+          atomicExch(p.sync, 1u);
+          break;
+        }
         const uint32_t bytes = cur.bytes();
         mbar_arrive_expect_tx(&full[slot], bytes);
         bulk_g2s_evict_first(ring + (size_t)slot * kSB, cur.src(), bytes, &full[slot], pol);
@@ -328,6 +388,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           par ^= 1u;
         }
       }
+      // every copy issued has landed before the CTA may exit (these waits
+      // only block if an earlier bounded wait gave up)
+      for (int sl = 0; sl < RING; ++sl)
+        if (gs > sl) bwait(&full[sl], (uint32_t)(((gs - 1 - sl) / RING) & 1), dl);
     }
     return;
   }
@@ -336,7 +400,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int ct = tid;
   const int Gq = p.nh / p.nkv;
   const int half = p.hd >> 1;
-  const bf16* X = reinterpret_cast<const bf16*>(p.x);
+  const Poll pl{dl, p.sync, p.err};
   long long gs = 0;    // weight stages consumed
   int c_slot = 0;      // ring slot and parity of the next stage
   uint32_t c_par = 0;
@@ -345,11 +409,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   long long best_i = LLONG_MAX;
 
   // The rows of the residual stream this CTA owns in the o and down phases,
-  // kept here between its epilogues (x in global memory is the copy the
-  // RMSNorm prologues read).
+  // kept here between its epilogues.
   {
-    const int r0 = (int)((long long)bid * p.H / G), r1 = (int)((long long)(bid + 1) * p.H / G);
-    const bf16* src = X;
+    const int units = p.H / 2;
+    const int r0 = (int)((long long)bid * units / G) * 2, r1 = (int)((long long)(bid + 1) * units / G) * 2;
+    const bf16* src = reinterpret_cast<const bf16*>(p.x);
     if (p.embed_in) {
       long long id = __ldcg(p.ids);
       if (id < 0 || id >= p.V) id = 0;
@@ -362,15 +426,27 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int i = 0; i < NCH; ++i) nwr[i] = __ldg(reinterpret_cast<const uint4*>(nw) + lane + 32 * i);
   };
-  // xr = bf16(rmsnorm(src) * nw): every warp normalises the whole vector itself.
-  auto norm_regs = [&](const bf16* src, const uint4 (&nwr)[NCH], float (&xr)[NCH][8]) {
+  // the phase's input vector into xbuf: from tagged words (bf16 pairs) ...
+  auto stage_tagged = [&](const uint64_t* ll, int nwords, uint32_t tag) {
+    for (int v = ct; v < nwords / 2; v += kCT) reinterpret_cast<uint2*>(xbuf)[v] = pl.get2(ll + 2 * v, tag);
+    csync();
+  };
+  // ... or from plain bf16 memory
+  auto stage_plain = [&](const bf16* src, int n) {
+    for (int c = ct; c < n / 8; c += kCT) reinterpret_cast<uint4*>(xbuf)[c] = __ldcg(reinterpret_cast<const uint4*>(src) + c);
+    csync();
+  };
+  // xr = this lane's pieces of xbuf, bf16(rmsnorm(xbuf) * nw) if nw is given:
+  // every warp normalises the whole vector itself.
+  auto input_regs = [&](bool norm, const uint4 (&nwr)[NCH], float (&xr)[NCH][8]) {
     float ss = 0.f;
 #pragma unroll
     for (int i = 0; i < NCH; ++i) {
-      unpack16<bf16>(__ldcg(reinterpret_cast<const uint4*>(src) + lane + 32 * i), xr[i]);
+      unpack16<bf16>(reinterpret_cast<const uint4*>(xbuf)[lane + 32 * i], xr[i]);
 #pragma unroll
       for (int e = 0; e < 8; ++e) ss = fmaf(xr[i][e], xr[i][e], ss);
     }
+    if (!norm) return;
     ss = warp_sum(ss);
     const float inv = rsqrtf(ss / (float)(NCH * 256) + p.eps);
 #pragma unroll
@@ -393,7 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         c_par ^= 1u;
       }
       const int n = min(pw.rs, pw.r1 - r);
-      if (!bwait(&full[slot], par, dl) && lane == 0) atomicOr(p.err, 2);
+      if (!bwait(&full[slot], par, dl, p.sync) && lane == 0) atomicOr(p.err, 2);
       const uint8_t* st = ring + (size_t)slot * kSB;
       for (int rr = warp; rr < n; rr += kCW) {
         const uint4* wrow = reinterpret_cast<const uint4*>(st + (size_t)rr * pw.K * 2);
@@ -433,7 +509,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         c_slot = 0;
         c_par ^= 1u;
       }
-      if (!bwait(&full[slot], par, dl) && lane == 0) atomicOr(p.err, 2);
+      if (!bwait(&full[slot], par, dl, p.sync) && lane == 0) atomicOr(p.err, 2);
       const uint4* wrow = reinterpret_cast<const uint4*>(ring + (size_t)slot * kSB) + warp * cpw;
       float a[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -453,7 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
 
   // ---- attention work items: (kv head, split) pairs; a split spans at least
-  // two tiles (one per warp group) and its range follows from the length.
+  // two tiles and its range follows from the length.
   struct AItem {
     int gq, split, ntiles, tps, t0, t1, nact;
   };
@@ -491,7 +567,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     phase_w(p, layers, ph, bid, G, pw);
     unsigned long long* ctr = p.ctrace ? p.ctrace + ((size_t)ph * G + bid) * 4 : nullptr;
     if (ctr && ct == 0) ctr[0] = gtimer();
-    uint4 nwr[NCH];    // the RMSNorm weight pieces of this phase (loaded before its wait)
+    uint4 nwr[NCH];    // the RMSNorm weight pieces of this phase (loaded before its input)
     float xr[NCH][8];  // short-row phases: this lane's pieces lane + 32 i of the input vector
 
     // ---- what does not depend on the previous phase, before waiting for it
@@ -504,17 +580,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if ((i & 1) == 0 && n / p.hd < p.nh + p.nkv)
           ecs[i >> 1] = __ldg(p.rope + (size_t)pos * half + ((n % p.hd) >> 1));
       }
-      // the first two tiles of this CTA's first attention item of the layer;
-      // the tile holding the new position is patched once its row exists
+      // the first two tiles of this CTA's first attention item of the layer
+      // (the tile holding the new position gets that row patched in later)
       if (ct == 0) {
-        s_flags[F_PRE] = 0;
-        s_flags[F_STALE] = -1;
+        s_flags[2] = 0;
         if (bid < aitems) {
           const AItem a = attn_item(bid);
           for (int q = 0; q < 2 && a.t0 + q < a.t1; ++q) {
             tile_issue(l, a.gq, a.t0 + q, ac + q);
-            if (a.t0 + q == a.ntiles - 1) s_flags[F_STALE] = ac + q;
-            s_flags[F_PRE] = q + 1;
+            s_flags[2] = q + 1;
           }
         }
       }
@@ -524,65 +598,55 @@ __global__ void __launch_bounds__(kThreads, 1)
       load_nw(p.final_norm, nwr);
     }
 
-    // ---- wait until every CTA has finished the previous phase
-    if (ph > 0) {
-      if (ct == 0) {
-        const unsigned target = (unsigned)G + (ph - 1 == p.stall_phase ? 1u : 0u);
-        unsigned* gave_up = p.sync + 5 * L + 1 + L * p.nkv;
-        if (!gwait(&p.sync[ph - 1], target, dl, gave_up)) {
-          atomicOr(p.err, 2);
-          atomicExch(gave_up, 1u);
-        }
-        __threadfence();
-        if (kind == PH_ATTN) fence_proxy_async_global();  // new K/V rows, read next by TMA
-      }
-      csync();
-    }
-    if (p.trace && ct == 0) {
-      const unsigned long long t = gtimer();
-      atomicMax(&p.trace[ph * 4 + 3], t);
-      if (bid == 0) p.trace[ph * 4 + 1] = t;
-    }
-    if (ctr && ct == 0) ctr[1] = gtimer();
-
+    // ---- the phase's input, then its weight stages
     if (kind == PH_ATTN) {
       // Tensor-core attention over each tile: warp (grp, wq) takes keys
       // [16 wq, 16 wq + 16) and output dims [64 grp, 64 grp + 64): scores
       // q_h . k_j by mma.sync (the kv head's query heads on M, keys on N, head
       // dims on K; both groups compute them), online softmax in fp32, P . V by
       // mma.sync (P in a bf16 high and low part) for the group's dims.  The
-      // four warps of a group are merged in shared memory, then the splits by
-      // the last split to finish.
+      // four warps of a group are merged in shared memory; the first split of
+      // a kv head then merges the other splits' partials and publishes.
       const int grp = warp >> 2, wq = warp & 3;
       const int fr = lane >> 2, fc = lane & 3;  // mma fragment coordinates
       const int mi = lane >> 3, mr = lane & 7;  // ldmatrix: lane addresses row mr of matrix mi
       const float sl2 = p.scale * kLog2e;
+      const uint32_t tq = rtag(ph - 1), ta = wtag(ph);
+      if (ctr && ct == 0) ctr[1] = gtimer();
       for (int item = bid; item < aitems; item += G) {
         const AItem a = attn_item(item);
         if (a.t0 >= a.t1) continue;
         const int nt = a.t1 - a.t0;
-        const int pre = item == bid ? s_flags[F_PRE] : 0;
-        const int stale = item == bid ? s_flags[F_STALE] : -1;
+        const int pre = item == bid ? s_flags[2] : 0;
         if (ct == 0)
           for (int q = pre; q < 2 && q < nt; ++q) tile_issue(l, a.gq, a.t0 + q, ac + q);
-        // the new K/V row (for a tile loaded before it was written): fetched
-        // now, stored into the tile once the tile has landed
-        uint4 nrow = make_uint4(0u, 0u, 0u, 0u);
-        if (stale >= 0 && warp == 0) {
-          const size_t off = (size_t)l * p.kv_layer_stride + ((size_t)a.gq * p.max_seq + pos) * kHD;
-          const bf16* src = reinterpret_cast<const bf16*>(lane < 16 ? p.kc : p.vc) + off;
-          nrow = __ldcg(reinterpret_cast<const uint4*>(src) + (lane & 15));
+        // q of the kv head's query heads and the new K/V row, from the tagged words
+        for (int v = ct; v < Gq * half / 2; v += kCT) {
+          const int hh = v / (half / 2), j = 2 * (v % (half / 2));
+          const uint2 d = pl.get2(p.ll.q + (size_t)(a.gq * Gq + hh) * half + j, tq);
+          bf16* qh = qst + hh * kHD;
+          qh[j] = __ushort_as_bfloat16((unsigned short)(d.x & 0xffffu));
+          qh[j + half] = __ushort_as_bfloat16((unsigned short)(d.x >> 16));
+          qh[j + 1] = __ushort_as_bfloat16((unsigned short)(d.y & 0xffffu));
+          qh[j + 1 + half] = __ushort_as_bfloat16((unsigned short)(d.y >> 16));
         }
+        for (int v = ct; v < half; v += kCT) {  // K pairs, then V pairs
+          const int sel = v / (half / 2), j = 2 * (v % (half / 2));
+          const uint2 d = pl.get2(p.ll.kv + (size_t)(sel * p.nkv + a.gq) * half + j, tq);
+          bf16* r = kvn + sel * kHD;
+          r[j] = __ushort_as_bfloat16((unsigned short)(d.x & 0xffffu));
+          r[j + half] = __ushort_as_bfloat16((unsigned short)(d.x >> 16));
+          r[j + 1] = __ushort_as_bfloat16((unsigned short)(d.y & 0xffffu));
+          r[j + 1 + half] = __ushort_as_bfloat16((unsigned short)(d.y >> 16));
+        }
+        csync();
         // A fragments of the query heads (bf16, unscaled); rows fr >= Gq are zero
         uint32_t qa[8][2];
-        {
-          const unsigned* qrow = reinterpret_cast<const unsigned*>(
-              reinterpret_cast<const bf16*>(p.qb) + (size_t)(a.gq * Gq + (fr < Gq ? fr : 0)) * kHD);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            qa[kk][0] = fr < Gq ? __ldcg(qrow + 8 * kk + fc) : 0u;
-            qa[kk][1] = fr < Gq ? __ldcg(qrow + 8 * kk + fc + 4) : 0u;
-          }
+        for (int kk = 0; kk < 8; ++kk) {
+          const bf16* qrow = qst + (fr < Gq ? fr : 0) * kHD + 16 * kk + 2 * fc;
+          qa[kk][0] = fr < Gq ? *reinterpret_cast<const uint32_t*>(qrow) : 0u;
+          qa[kk][1] = fr < Gq ? *reinterpret_cast<const uint32_t*>(qrow + 8) : 0u;
         }
         float o[8][4];
 #pragma unroll
@@ -593,11 +657,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int t = a.t0 + i;
           if (!bwait(&abar[stg], (uint32_t)((li >> 1) & 1), dl) && lane == 0) atomicOr(p.err, 2);
           uint8_t* tk = tiles + (size_t)stg * 2 * kTile;
-          if (li == stale) {
+          if (t == a.ntiles - 1) {
+            // the tile holding the new position: its row comes from the
+            // published K/V (the cache row may have been read before it existed)
             if (warp == 0) {
               const int r = pos - t * kAT, c = lane & 15;
               uint8_t* dst = tk + (lane < 16 ? 0 : kTile) + (c >> 3) * 8192 + r * 128 + (((c & 7) ^ (r & 7)) << 4);
-              *reinterpret_cast<uint4*>(dst) = nrow;
+              *reinterpret_cast<uint4*>(dst) = reinterpret_cast<const uint4*>(kvn + (lane < 16 ? 0 : kHD))[c];
               fence_proxy_async_smem();
             }
             csync();
@@ -651,8 +717,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             ph_[e] = __bfloat162float(__float2bfloat16_rn(pr[e]));
             pl_[e] = pr[e] - ph_[e];
           }
-          const uint32_t pa0 = pack_bf16x2(ph_[0], ph_[1]), pa2 = pack_bf16x2(ph_[2], ph_[3]);
-          const uint32_t pb0 = pack_bf16x2(pl_[0], pl_[1]), pb2 = pack_bf16x2(pl_[2], pl_[3]);
+          const uint32_t pa0 = bf2_bits(ph_[0], ph_[1]), pa2 = bf2_bits(ph_[2], ph_[3]);
+          const uint32_t pb0 = bf2_bits(pl_[0], pl_[1]), pb2 = bf2_bits(pl_[2], pl_[3]);
           // positions past the sequence hold stale cache rows (possibly not
           // finite): their V entries are zeroed, as 0 * inf would poison the sum
           const uint32_t vm0 = (kb < alen ? 0x0000ffffu : 0u) | (kb + 1 < alen ? 0xffff0000u : 0u);
@@ -681,8 +747,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ac += nt;
 
-        // ---- the four warps of each group (max, sum, unnormalised output), merged;
-        // the tile buffers are free now (every tile of the item was waited on)
+        // ---- the four warps of each group (max, sum, unnormalised output),
+        // merged; the tile buffers are free now (every tile of the item was
+        // waited on)
         float* Ow = reinterpret_cast<float*>(tiles);  // [kCW][kAGMax][64]
         if (fr < Gq) {
 #pragma unroll
@@ -697,107 +764,72 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         csync();
-        const bool direct = a.nact == 1;
-        for (int i = ct; i < Gq * kHD; i += kCT) {
-          const int hh = i / kHD, d = i % kHD, w0 = 4 * (d >> 6);
+        // thread i takes dims (2 dp, 2 dp + 1) of head hh
+        for (int i = ct; i < Gq * half; i += kCT) {
+          const int hh = i / half, dp = i % half, d = 2 * dp, w0 = 4 * (d >> 6);
           float M = -INFINITY;
 #pragma unroll
           for (int w = w0; w < w0 + 4; ++w) M = fmaxf(M, mlw[(w * kAGMax + hh) * 2]);
           const float Ms = M == -INFINITY ? 0.f : M;
-          float O = 0.f, Ls = 0.f;
+          float O0 = 0.f, O1 = 0.f, Ls = 0.f;
 #pragma unroll
           for (int w = w0; w < w0 + 4; ++w) {
             const float e = exp2f(mlw[(w * kAGMax + hh) * 2] - Ms);
-            O = fmaf(e, Ow[((size_t)w * kAGMax + hh) * 64 + (d & 63)], O);
+            const float* ow = Ow + ((size_t)w * kAGMax + hh) * 64 + (d & 63);
+            O0 = fmaf(e, ow[0], O0);
+            O1 = fmaf(e, ow[1], O1);
             Ls = fmaf(e, mlw[(w * kAGMax + hh) * 2 + 1], Ls);
           }
-          if (direct) {
-            reinterpret_cast<bf16*>(p.att)[(size_t)(a.gq * Gq + hh) * kHD + d] =
-                __float2bfloat16_rn(Ls > 0.f ? O / Ls : 0.f);
+          uint64_t* pbase = p.ll.part + ((size_t)(a.gq * kSplitMax + a.split) * Gq + hh) * (kHD + 2);
+          if (a.split > 0) {  // a partial for the first split of this kv head
+            ll_put2(pbase + d, __float_as_uint(O0), __float_as_uint(O1), ta);
+            if (dp == 0) ll_put2(pbase + kHD, __float_as_uint(M), __float_as_uint(Ls), ta);
           } else {
-            const size_t pidx = (size_t)(a.gq * Gq + hh) * p.nsplit + a.split;
-            p.part_o[pidx * kHD + d] = O;
-            if (d == 0) {
-              p.part_ml[2 * pidx] = M;
-              p.part_ml[2 * pidx + 1] = Ls;
+            // the first split merges the others in split order:
+            // o = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s
+            for (int sp = 1; sp < a.nact; ++sp) {
+              const uint64_t* ob = p.ll.part + ((size_t)(a.gq * kSplitMax + sp) * Gq + hh) * (kHD + 2);
+              const uint2 ml = pl.get2(ob + kHD, rtag(ph));
+              const uint2 ov = pl.get2(ob + d, rtag(ph));
+              const float ms = __uint_as_float(ml.x), lsp = __uint_as_float(ml.y);
+              const float Mn = fmaxf(M, ms);
+              const float ea = exp2f(M - Mn), eb = exp2f(ms - Mn);
+              O0 = O0 * ea + __uint_as_float(ov.x) * eb;
+              O1 = O1 * ea + __uint_as_float(ov.y) * eb;
+              Ls = Ls * ea + lsp * eb;
+              M = Mn;
             }
+            const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+            ll_put(p.ll.att + (size_t)(a.gq * Gq + hh) * half + dp, bf2_bits(O0 * inv, O1 * inv), ta);
           }
         }
         fence_proxy_async_smem();  // the tile buffer is a TMA destination again later
-        if (!direct) {
-          // ---- the last of the nact splits of this kv head merges them:
-          // o = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s, in split order
-          __threadfence();
-          csync();
-          if (ct == 0) {
-            unsigned* ticket = p.sync + 5 * L + 1 + l * p.nkv + a.gq;
-            s_flags[F_MERGE] = atomicAdd(ticket, 1u) == (unsigned)a.nact - 1;
-          }
-          csync();
-          if (s_flags[F_MERGE]) {
-            __threadfence();
-            for (int i = ct; i < Gq * a.nact; i += kCT) {
-              const int hh = i / a.nact, sp = i % a.nact;
-              const size_t pidx = (size_t)(a.gq * Gq + hh) * p.nsplit + sp;
-              mraw[hh * kSplitMax + sp] = __ldcg(p.part_ml + 2 * pidx);
-              wts[hh * kSplitMax + sp] = __ldcg(p.part_ml + 2 * pidx + 1);
-            }
-            csync();
-            if (ct < Gq) {
-              float Mx = -INFINITY;
-              for (int sp = 0; sp < a.nact; ++sp) Mx = fmaxf(Mx, mraw[ct * kSplitMax + sp]);
-              const float Ms = Mx == -INFINITY ? 0.f : Mx;
-              float den = 0.f;
-              for (int sp = 0; sp < a.nact; ++sp) {
-                const float e = exp2f(mraw[ct * kSplitMax + sp] - Ms);
-                mraw[ct * kSplitMax + sp] = e;
-                den = fmaf(wts[ct * kSplitMax + sp], e, den);
-              }
-              const float inv = den > 0.f ? 1.f / den : 0.f;
-              for (int sp = 0; sp < a.nact; ++sp) wts[ct * kSplitMax + sp] = mraw[ct * kSplitMax + sp] * inv;
-            }
-            csync();
-            for (int e = ct; e < Gq * kHD; e += kCT) {
-              const int hh = e / kHD, d = e % kHD;
-              const float* po = p.part_o + ((size_t)(a.gq * Gq + hh) * p.nsplit) * kHD + d;
-              const float* wv = wts + hh * kSplitMax;
-              float o0 = 0.f, o1 = 0.f;
-              int sp = 0;
-              for (; sp + 1 < a.nact; sp += 2) {
-                o0 = fmaf(wv[sp], __ldcg(po + (size_t)sp * kHD), o0);
-                o1 = fmaf(wv[sp + 1], __ldcg(po + (size_t)(sp + 1) * kHD), o1);
-              }
-              if (sp < a.nact) o0 = fmaf(wv[sp], __ldcg(po + (size_t)sp * kHD), o0);
-              reinterpret_cast<bf16*>(p.att)[(size_t)(a.gq * Gq + hh) * kHD + d] = __float2bfloat16_rn(o0 + o1);
-            }
-          }
-        }
         csync();
       }
     } else if (kind == PH_DOWN) {
       float xs[NQ][8];  // this lane's pieces of the warp's column slice of s
       const int cpw = pw.K / 8 / kCW;
-      const uint4* sv = reinterpret_cast<const uint4*>(p.s) + warp * cpw;
+      const uint32_t tg = rtag(ph - 1);
 #pragma unroll
       for (int q = 0; q < NQ; ++q) {
-        if (lane + 32 * q < cpw) {
-          unpack16<bf16>(__ldcg(sv + lane + 32 * q), xs[q]);
+        const int c = lane + 32 * q;
+        if (c < cpw) {
+          const uint64_t* w = p.ll.s + (size_t)(warp * cpw + c) * 4;
+          const uint2 a = pl.get2(w, tg), b = pl.get2(w + 2, tg);
+          unpack16<bf16>(make_uint4(a.x, a.y, b.x, b.y), xs[q]);
         } else {
 #pragma unroll
           for (int e = 0; e < 8; ++e) xs[q][e] = 0.f;
         }
       }
+      if (ctr && ct == 0) ctr[1] = gtimer();
       consume_long(pw, xs);
     } else {  // the short-row phases: q/k/v, o, gate/up, lm_head
-      if (kind == PH_O) {
-#pragma unroll
-        for (int i = 0; i < NCH; ++i)
-          unpack16<bf16>(__ldcg(reinterpret_cast<const uint4*>(p.att) + lane + 32 * i), xr[i]);
-      } else {
-        const bf16* src = X;
-        if (kind == PH_QKV && l == 0 && p.embed_in) {
-          // layer 0 normalises the embedding row directly.  An id outside the
-          // vocabulary sets bit 0 of the error word and reads row 0.
+      if (kind == PH_QKV && l == 0) {
+        // layer 0: the embedding row (an id outside the vocabulary sets bit 0 of
+        // the error word and reads row 0), or the caller's input
+        const bf16* src = reinterpret_cast<const bf16*>(p.x);
+        if (p.embed_in) {
           long long id = __ldcg(p.ids);
           if (id < 0 || id >= p.V) {
             if (ct == 0 && bid == 0) atomicOr(p.err, 1);
@@ -805,14 +837,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           src = reinterpret_cast<const bf16*>(p.embed) + (size_t)id * p.H;
         }
-        norm_regs(src, nwr, xr);
+        stage_plain(src, p.H);
+      } else if (kind == PH_O) {
+        stage_tagged(p.ll.att, p.qd / 2, rtag(ph - 1));
+      } else {  // x from the previous o or down phase
+        stage_tagged(p.ll.x, p.H / 2, rtag(ph - 1));
       }
+      if (ctr && ct == 0) ctr[1] = gtimer();
+      input_regs(kind != PH_O, nwr, xr);
       consume_short(pw, kind == PH_HEAD, xr);
     }
 
     // ---- phase epilogue from the parked row results and staged operands
     csync();
     if (ctr && ct == 0) ctr[2] = gtimer();
+    const uint32_t tw = wtag(ph);
     if (kind == PH_QKV) {
       const size_t loff = (size_t)l * p.kv_layer_stride;
       for (int i = ct; 2 * i < pw.r1 - pw.r0; i += kCT) {
@@ -820,42 +859,55 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int hs = n / p.hd, j = (n % p.hd) >> 1;
         const float va = round_st<bf16>(yrow[2 * i] + ebias[2 * i]);
         const float vb = round_st<bf16>(yrow[2 * i + 1] + ebias[2 * i + 1]);
+        bf16 ra, rb;
         if (hs < p.nh + p.nkv) {
           const float2 cs = ecs[i];
-          const bf16 ra = __float2bfloat16_rn(va * cs.x - vb * cs.y);
-          const bf16 rb = __float2bfloat16_rn(vb * cs.x + va * cs.y);
-          bf16* dst = hs < p.nh ? reinterpret_cast<bf16*>(p.qb) + (size_t)hs * p.hd
-                                : reinterpret_cast<bf16*>(p.kc) + loff + ((size_t)(hs - p.nh) * p.max_seq + pos) * p.hd;
+          ra = __float2bfloat16_rn(va * cs.x - vb * cs.y);
+          rb = __float2bfloat16_rn(vb * cs.x + va * cs.y);
+        } else {
+          ra = __float2bfloat16_rn(va);
+          rb = __float2bfloat16_rn(vb);
+        }
+        if (hs < p.nh) {
+          ll_put(p.ll.q + (size_t)hs * half + j, bf2_bits(ra, rb), tw);
+        } else {
+          const int kvh = hs - p.nh;  // 0 .. nkv - 1: K heads, nkv .. 2 nkv - 1: V heads
+          bf16* dst = reinterpret_cast<bf16*>(kvh < p.nkv ? p.kc : p.vc) + loff +
+                      ((size_t)(kvh % p.nkv) * p.max_seq + pos) * p.hd;
           dst[j] = ra;
           dst[j + half] = rb;
-        } else {
-          bf16* dst = reinterpret_cast<bf16*>(p.vc) + loff +
-                      ((size_t)(hs - p.nh - p.nkv) * p.max_seq + pos) * p.hd;
-          dst[j] = __float2bfloat16_rn(va);
-          dst[j + half] = __float2bfloat16_rn(vb);
+          ll_put(p.ll.kv + (size_t)kvh * half + j, bf2_bits(ra, rb), tw);
         }
       }
-      fence_proxy_async_global();  // attention may read the new K/V rows by TMA
     } else if (kind == PH_O || kind == PH_DOWN) {
       bf16* xw = reinterpret_cast<bf16*>(p.x);
-      for (int i = ct; i < pw.r1 - pw.r0; i += kCT) {
-        float y;
+      for (int i = ct; 2 * i < pw.r1 - pw.r0; i += kCT) {
+        float y0, y1;
         if (kind == PH_O) {
-          y = yrow[i];
+          y0 = yrow[2 * i];
+          y1 = yrow[2 * i + 1];
         } else {
-          y = 0.f;
+          y0 = y1 = 0.f;
 #pragma unroll
-          for (int w = 0; w < kCW; ++w) y += part[w * kDMax + i];
+          for (int w = 0; w < kCW; ++w) {
+            y0 += part[w * kDMax + 2 * i];
+            y1 += part[w * kDMax + 2 * i + 1];
+          }
         }
-        const bf16 xn = __float2bfloat16_rn(xres[i] + round_st<bf16>(y));
-        xw[pw.r0 + i] = xn;
-        xres[i] = __bfloat162float(xn);
+        const bf16 x0 = __float2bfloat16_rn(xres[2 * i] + round_st<bf16>(y0));
+        const bf16 x1 = __float2bfloat16_rn(xres[2 * i + 1] + round_st<bf16>(y1));
+        const int n = pw.r0 + 2 * i;
+        xw[n] = x0;
+        xw[n + 1] = x1;
+        xres[2 * i] = __bfloat162float(x0);
+        xres[2 * i + 1] = __bfloat162float(x1);
+        ll_put(p.ll.x + n / 2, bf2_bits(x0, x1), tw);
       }
     } else if (kind == PH_GU) {
-      bf16* sw = reinterpret_cast<bf16*>(p.s);
-      for (int i = ct; 2 * i < pw.r1 - pw.r0; i += kCT) {
-        const float gv = round_st<bf16>(yrow[2 * i]), uv = round_st<bf16>(yrow[2 * i + 1]);
-        sw[(pw.r0 >> 1) + i] = __float2bfloat16_rn(silu_mul(gv, uv));
+      for (int i = ct; 4 * i < pw.r1 - pw.r0; i += kCT) {
+        const float s0 = silu_mul(round_st<bf16>(yrow[4 * i]), round_st<bf16>(yrow[4 * i + 1]));
+        const float s1 = silu_mul(round_st<bf16>(yrow[4 * i + 2]), round_st<bf16>(yrow[4 * i + 3]));
+        ll_put(p.ll.s + pw.r0 / 4 + i, bf2_bits(s0, s1), tw);
       }
     } else if (kind == PH_HEAD) {
       if (lane == 0) {
@@ -871,16 +923,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             bv = amv[w];
             bi = ami[w];
           }
-        p.am_val[bid] = bv;
-        p.am_idx[bid] = bi;
+        ll_put2(p.ll.am + 2 * bid, __float_as_uint(bv), (uint32_t)bi, tw);
       }
     }
-
-    // ---- this CTA is done with the phase
-    csync();
     if (ct == 0) {
-      __threadfence();
-      s_flags[F_LAST] = atom_add_release(&p.sync[ph], 1u) == (unsigned)G - 1 && ph == nph - 1;
       if (ctr) ctr[3] = gtimer();
       if (p.trace) {
         const unsigned long long t = gtimer();
@@ -890,34 +936,54 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
-  // ---- drain: every copy this CTA issued has landed before it exits (the
-  // waits only block if an earlier bounded wait gave up)
+  // ---- drain: every attention tile this CTA issued has landed before it
+  // exits (the producer drains the weight ring)
   if (ct == 0) {
-    for (int sl = 0; sl < RING; ++sl)
-      if (gs > sl) bwait(&full[sl], (uint32_t)(((gs - 1 - sl) / RING) & 1), dl);
     for (int st = 0; st < 2; ++st)
       if (ac > st) bwait(&abar[st], (uint32_t)(((ac - 1 - st) / 2) & 1), dl);
   }
-  csync();
 
-  // ---- the last arrival of the last phase wraps up the step: the token
-  // (argmax over the CTAs' partials) and the length
-  if (s_flags[F_LAST] && ct == 0) {
-    __threadfence();
+  // ---- CTA 0 wraps up the step: the token (argmax over the CTAs' partials,
+  // which the order of the pairs alone decides), the length, the step counter
+  if (bid == 0) {
     if (p.run_head) {
       float bv = -INFINITY;
       long long bi = LLONG_MAX;
-      for (int b = 0; b < G; ++b) {
-        const float v = __ldcg(p.am_val + b);
-        const long long i = __ldcg(reinterpret_cast<const long long*>(p.am_idx) + b);
-        if (am_better(v, i, bv, bi)) {
-          bv = v;
-          bi = i;
+      for (int c = ct; c < G; c += kCT) {
+        const uint2 d = pl.get2(p.ll.am + 2 * c, rtag(nph - 1));
+        if (am_better(__uint_as_float(d.x), (long long)d.y, bv, bi)) {
+          bv = __uint_as_float(d.x);
+          bi = (long long)d.y;
         }
       }
-      p.next[0] = bi;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const long long oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (am_better(ov, oi, bv, bi)) {
+          bv = ov;
+          bi = oi;
+        }
+      }
+      csync();  // amv / ami are free again
+      if (lane == 0) {
+        amv[warp] = bv;
+        ami[warp] = bi;
+      }
+      csync();
+      if (ct == 0) {
+        for (int w = 0; w < kCW; ++w)
+          if (am_better(amv[w], ami[w], bv, bi)) {
+            bv = amv[w];
+            bi = ami[w];
+          }
+        p.next[0] = bi;
+      }
     }
-    p.lens[0] += 1;
+    if (ct == 0) {
+      p.lens[0] += 1;
+      *p.epoch += 1u;
+    }
   }
 }
 
@@ -925,25 +991,63 @@ __global__ void __launch_bounds__(kThreads, 1)
 namespace {
 constexpr int kNCH = 6;  // H = 1536
 constexpr int kNQ = 5;   // ceil(I / 8 / kCW / 32) for I = 8960
+
+// the tagged buffers, each starting on a 16-byte boundary
+struct LLSizes {
+  size_t x, q, kv, att, s, part, am;
+};
+LLSizes ll_sizes(int H, int I, int nh, int nkv, int hd, int grid) {
+  auto even = [](size_t n) { return (n + 1) / 2 * 2; };
+  LLSizes z;
+  z.x = even((size_t)H / 2);
+  z.q = even((size_t)nh * hd / 2);
+  z.kv = even((size_t)2 * nkv * hd / 2);
+  z.att = even((size_t)nh * hd / 2);
+  z.s = even((size_t)I / 2);
+  z.part = even((size_t)nkv * kSplitMax * (nh / nkv) * (hd + 2));
+  z.am = (size_t)2 * grid;
+  return z;
+}
 }  // namespace
+
+size_t sdecode_ll_words(int H, int I, int nh, int nkv, int hd, int grid) {
+  const LLSizes z = ll_sizes(H, I, nh, nkv, hd, grid);
+  return z.x + z.q + z.kv + z.att + z.s + z.part + z.am;
+}
+
+SDecodeLL sdecode_ll_carve(uint64_t* base, int H, int I, int nh, int nkv, int hd, int grid) {
+  const LLSizes z = ll_sizes(H, I, nh, nkv, hd, grid);
+  SDecodeLL b;
+  b.x = base;
+  b.q = b.x + z.x;
+  b.kv = b.q + z.q;
+  b.att = b.kv + z.kv;
+  b.s = b.att + z.att;
+  b.part = b.s + z.s;
+  b.am = b.part + z.part;
+  return b;
+}
 
 bool sdecode_supported(int H, int I, int V, int nh, int nkv, int hd, int qkvd, int qd) {
   if (hd != kHD || nkv <= 0 || nh % nkv != 0 || nh / nkv > kAGMax || V <= 0) return false;
-  if (H != kNCH * 256 || qd != H || qkvd % 2 != 0) return false;
+  if (H != kNCH * 256 || qd != H || H > kHMax || qkvd % 2 != 0) return false;
   if (I % (8 * kCW) != 0 || (I / 8 / kCW + 31) / 32 != kNQ || I * 2 > kSB || I * 2 <= kSB / 2)
     return false;
   return true;
 }
 
-// phase counters [5L + 1], merge tickets [L][nkv], the launch's give-up word
-size_t sdecode_sync_words(int L, int nkv) { return (size_t)5 * L + 1 + (size_t)L * nkv + 1; }
+size_t sdecode_sync_words() { return 4; }
 
-int sdecode_default_ring() { return 6; }
+int sdecode_max_ring(int L) {
+  for (int ring = 8; ring >= 2; --ring)
+    if (slayout(ring, L).total <= kSmemMax) return ring;
+  return 0;
+}
 
 q2_status launch_sdecode(const SDecode& p, const CUtensorMap& kmap, const CUtensorMap& vmap,
                          cudaStream_t st) {
   if (!sdecode_supported(p.H, p.I, p.V, p.nh, p.nkv, p.hd, p.qkvd, p.qd) || p.nsplit < 1 ||
-      p.nsplit > kSplitMax || p.ring < 2 || p.L < 1 || p.L > kLMax) {
+      p.nsplit > kSplitMax || p.ring < 2 || p.L < 1) {
     set_error("streaming decode: unsupported shape");
     return Q2_ERR_SHAPE;
   }
@@ -955,8 +1059,8 @@ q2_status launch_sdecode(const SDecode& p, const CUtensorMap& kmap, const CUtens
   const int G = num_sms();
   // rows per CTA of the phases whose row results and operands sit in shared memory
   const long long qkv_rows = (long long)(p.qkvd / 2 + G - 1) / G * 2;
-  const long long gu_rows = (long long)(p.I + G - 1) / G * 2;
-  const long long o_rows = (p.H + G - 1) / G;
+  const long long gu_rows = (long long)(2 * p.I / 4 + G - 1) / G * 4;
+  const long long o_rows = (long long)(p.H / 2 + G - 1) / G * 2;
   if (qkv_rows > kQMax || gu_rows > kYMax || o_rows > kYMax || o_rows > kDMax) {
     set_error("streaming decode: too many rows per CTA for this device");
     return Q2_ERR_SHAPE;

@@ -7,32 +7,40 @@
 // step from that bound is not the streaming itself but the fixed cost of each
 // dependency: the layer is a chain of five all-to-all steps (q/k/v, attention,
 // o, gate/up, down), each needing the whole output of the one before.  The
-// kernel therefore decouples the two:
+// kernel attacks both sides:
 //
 //  * a producer warp per CTA streams this CTA's rows of every weight matrix
 //    of the step -- layer by layer q/k/v, o, gate/up, down, then the lm_head
 //    -- through a ring of shared-memory slots (one bulk copy per slot of
 //    whole rows).  It waits only for free slots, never for a phase, so the
-//    weights of the next phases are already landing while the grid waits at a
-//    phase boundary or runs attention;
-//  * eight consumer warps run the phases in order, separated by grid-wide
-//    counters.  Each warp keeps the phase's input vector in registers (for
-//    the RMSNorm phases it normalises the whole vector itself: no block-level
-//    reduction), takes whole rows of a slot (rows of K = hidden) or a column
-//    slice of a row (the down rows), and parks the row results in shared
-//    memory; the phase's epilogue (bias + RoPE + KV append, residual add,
-//    SwiGLU, logits + argmax) runs once at the phase end from there.
+//    weights of the next phases are already landing while the consumers wait
+//    for a phase's input or run attention;
+//  * the phases exchange their outputs as tagged words: every 8-byte word
+//    holds 4 bytes of data and a 4-byte tag naming the step and the phase
+//    that wrote it, stored with one 8-byte store.  A reader polls the words
+//    it needs until each carries the tag it expects -- one store-to-load hop,
+//    with no fence, no grid barrier and no counter.  (Each phase needs the
+//    whole output of the previous one, so no CTA can get more than one phase
+//    ahead of another; that ordering is what makes every buffer reuse safe.)
+//  * eight consumer warps run the phases.  Each warp keeps the phase's input
+//    vector in registers (for the RMSNorm phases it normalises the whole
+//    vector itself), takes whole rows of a slot (rows of K = hidden) or a
+//    column slice of a row (the down rows), and parks the row results in
+//    shared memory; the phase's epilogue (bias + RoPE + KV append, residual
+//    add, SwiGLU, logits + argmax) runs once at the phase end from there.
 //
 // Phases (l = layer):
-//   QKV(l)  RMSNorm (layer 0: embedding gather) -> q/k/v rows, bias, RoPE,
-//           q out, K/V appended to the cache
-//   ATTN(l) split attention over the cache (K/V tiles by TMA), the splits of a
-//           kv head merged by the last of its CTAs
-//   O(l)    o rows, residual add
-//   GU(l)   RMSNorm -> gate/up row pairs, SwiGLU
+//   QKV(l)  RMSNorm (layer 0: embedding row) -> q/k/v rows, bias, RoPE; q and
+//           the new K/V row published, K/V appended to the cache
+//   ATTN(l) split attention over the cache (K/V tiles by TMA, the tile holding
+//           the new position patched with the published row); the first split
+//           of a kv head merges the others' partials and publishes the output
+//   O(l)    o rows, residual add (x published)
+//   GU(l)   RMSNorm -> gate/up row pairs, SwiGLU (s published)
 //   DOWN(l) down rows (each split over the warps by columns), residual add
-//   HEAD    final RMSNorm -> lm_head rows, fp32 logits, argmax (the last
-//           arrival reduces the CTAs' partials and advances the length)
+//   HEAD    final RMSNorm -> lm_head rows, fp32 logits, per-CTA argmax; CTA 0
+//           reduces the partials, writes the token and advances the length
+//           and the step counter
 // Every wait is bounded by a deadline on the global timer; a wait that runs
 // out sets bit 1 (value 2) of the error word and the step carries on (its
 // results are then undefined), so a broken dependency cannot hang the GPU.
@@ -47,6 +55,19 @@
 
 namespace q2 {
 
+// The tagged exchange buffers (8-byte words), carved from one allocation.
+struct SDecodeLL {
+  uint64_t* x;     // [H / 2]        residual stream, bf16 pairs (2i, 2i + 1)
+  uint64_t* q;     // [nh * hd / 2]  rotated q, head h word j = (q[j], q[j + hd/2])
+  uint64_t* kv;    // [2 * nkv * hd / 2] the new K row pairs, then the new V row pairs (same pairing)
+  uint64_t* att;   // [nh * hd / 2]  attention output, bf16 pairs (2i, 2i + 1)
+  uint64_t* s;     // [I / 2]        SwiGLU output, bf16 pairs
+  uint64_t* part;  // [nkv][split max][nh / nkv][hd + 2] fp32 split partials (o, then max, sum)
+  uint64_t* am;    // [grid][2]      per-CTA argmax (value bits, index)
+};
+size_t sdecode_ll_words(int H, int I, int nh, int nkv, int hd, int grid);
+SDecodeLL sdecode_ll_carve(uint64_t* base, int H, int I, int nh, int nkv, int hd, int grid);
+
 struct SDecode {
   const PLayer* layers;  // device array [L]
   int L, H, I, V, nh, nkv, hd, qkvd, qd;
@@ -58,38 +79,34 @@ struct SDecode {
   const void* lm_head;
   const void* final_norm;
   const int64_t* ids;    // [1]
-  void* x;               // residual stream [H] (bf16), sequence 0
-  void* qb;              // [qd] rotated q
-  void* att;             // [qd] merged attention output
-  void* s;               // [I] SwiGLU output
+  void* x;               // residual stream [H] (bf16), sequence 0: the input when embed_in = 0,
+                         // the output of the layers at the end
   void* kc;              // K / V cache [L][Bmax][nkv][max_seq][hd]
   void* vc;
   long long kv_layer_stride;
   const float2* rope;    // [max_seq][hd/2]
   int* lens;             // [Bmax]; sequence 0's length = the new token's position
-  float* part_o;         // [nh][nsplit][hd]
-  float* part_ml;        // [nh][nsplit][2]
+  SDecodeLL ll;          // tagged exchange buffers
+  unsigned* epoch;       // step counter (tags are unique per step and phase); advanced by CTA 0
   float* logits;         // [V]
-  float* am_val;         // [grid]
-  int64_t* am_idx;       // [grid]
   int64_t* next;         // [1]
-  unsigned* sync;        // [sdecode_sync_words(L, nkv)], zero at launch
-  unsigned long long* trace;  // optional [5L + 1][4] phase timestamps
+  unsigned* sync;        // [sdecode_sync_words()], zero at launch: [0] a wait of this launch gave up
+  unsigned long long* trace;   // optional [5L + 1][4] phase timestamps
   unsigned long long* ctrace;  // optional [5L + 1][grid][4] per-CTA timestamps: phase entered,
-                               // previous phase seen complete, stages consumed, arrival
+                               // input complete, phase work done, outputs published
   int* err;              // bit 0 (1): id outside the vocabulary; bit 1 (2): a wait ran out
   int ring;              // weight ring slots
   int l2_ahead;          // weight slots the producer pulls into L2 ahead of the ring (0: none)
   unsigned long long deadline_ns;  // bound of every wait
-  int stall_phase;       // test hook: the counter of this phase needs one arrival more than
-                         // the grid makes, so its waits run out (-1: none)
+  int stall_phase;       // test hook: the output of this phase never carries the tag its
+                         // readers wait for, so their waits run out (-1: none)
 };
 
 bool sdecode_supported(int H, int I, int V, int nh, int nkv, int hd, int qkvd, int qd);
-// phase counters, per (layer, kv head) merge tickets, and one word a wait
-// that ran out sets so the launch's other grid waits give up at once
-size_t sdecode_sync_words(int L, int nkv);
-int sdecode_default_ring();
+constexpr int kSDecodeSplitMax = 64;
+size_t sdecode_sync_words();
+// The deepest weight ring whose shared-memory plan fits for L layers (0: none).
+int sdecode_max_ring(int L);
 q2_status launch_sdecode(const SDecode& p, const CUtensorMap& kmap, const CUtensorMap& vmap,
                          cudaStream_t st);
 
