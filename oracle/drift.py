@@ -10,6 +10,11 @@ the free-running tolerances of the tests are derived from it.
 
     python -m oracle.drift prompt  [--tokens 6]          # prefill of a short prompt
     python -m oracle.drift cache   [--context 32768]     # one token over an N(0,1) cache
+    python -m oracle.drift layer   [--tokens 128] [--layer 0]
+        # one decoder layer on the prompt's layer input (the embedding rows for
+        # layer 0): the elementwise scaled error max |a - b| / max(|b|, rms(b))
+        # and the relative norm error of the layer output (the layer bound's
+        # two measures)
 
 Each side runs in its own process (the library variant is chosen at import).
 """
@@ -22,11 +27,21 @@ import sys
 _ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def _logits(mode: str, n: int) -> list:
+def _logits(mode: str, n: int, layer: int = 0) -> list:
     sys.path.insert(0, _ROOT)
+    import dataclasses
     import synth
     import oracle
     shape = synth.QWEN2_1P5B
+    if mode == "layer":
+        w = synth.model_weights(shape, 1003)
+        x = oracle.embedding(synth.prompt_ids(shape, n, 1003 + 500), w[("embed", -1)])
+        for l in range(layer + 1):
+            one = dataclasses.replace(shape, n_layers=1)
+            om = oracle.OracleModel(one, max_seq=n)
+            om.load({(k, 0): t for (k, ll), t in w.items() if ll == l})
+            x = om.forward_hidden(0, x)
+        return x.double().reshape(-1).tolist()
     if mode == "prompt":
         w = synth.model_weights(shape, 1003)
         om = oracle.OracleModel(shape, max_seq=n + 8)
@@ -48,26 +63,37 @@ def _logits(mode: str, n: int) -> list:
 
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
-    ap.add_argument("mode", choices=["prompt", "cache"])
+    ap.add_argument("mode", choices=["prompt", "cache", "layer"])
     ap.add_argument("--tokens", type=int, default=6)
     ap.add_argument("--context", type=int, default=32768)
+    ap.add_argument("--layer", type=int, default=0)
     ap.add_argument("--child", action="store_true", help=argparse.SUPPRESS)
     a = ap.parse_args()
-    n = a.tokens if a.mode == "prompt" else a.context
+    n = a.context if a.mode == "cache" else a.tokens
     if a.child:
-        json.dump(_logits(a.mode, n), sys.stdout)
+        json.dump(_logits(a.mode, n, a.layer), sys.stdout)
         return
-    out = []
-    for f32 in ("0", "1"):
+    procs = []
+    for f32 in ("0", "1"):  # the two builds side by side
         env = dict(os.environ, ORACLE_FP32_ACCUMULATION=f32)
-        p = subprocess.run([sys.executable, "-m", "oracle.drift", a.mode, "--tokens", str(a.tokens),
-                            "--context", str(a.context), "--child"], cwd=_ROOT, env=env,
-                           capture_output=True, text=True, check=True)
-        out.append(json.loads(p.stdout))
+        procs.append(subprocess.Popen([sys.executable, "-m", "oracle.drift", a.mode, "--tokens", str(a.tokens),
+                                       "--context", str(a.context), "--layer", str(a.layer), "--child"],
+                                      cwd=_ROOT, env=env, stdout=subprocess.PIPE, text=True))
+    out = []
+    for p in procs:
+        o, _ = p.communicate()
+        if p.returncode != 0:
+            raise SystemExit(p.returncode)
+        out.append(json.loads(o))
     import torch
     r, g = torch.tensor(out[0], dtype=torch.float64), torch.tensor(out[1], dtype=torch.float64)
     res = {"mode": a.mode, "n": n, "max_abs": float((g - r).abs().max()),
            "cosine": float(torch.nn.functional.cosine_similarity(g, r, dim=0))}
+    if a.mode == "layer":
+        scale = torch.maximum(r.abs(), r.pow(2).mean().sqrt().expand_as(r))
+        res["layer"] = a.layer
+        res["max_scaled"] = float(((g - r).abs() / scale).max())
+        res["rel_norm"] = float((g - r).norm() / r.norm())
     print(json.dumps(res))
 
 

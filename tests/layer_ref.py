@@ -119,3 +119,13 @@ def prefill(pool, shape, weights: Dict, ids: torch.Tensor, max_seq: int, keep_la
         caches.append((kc, vc))
     nxt, logits = head(pool, shape, weights[("final_norm", -1)], weights[("lm_head", -1)], x[T - 1:T])
     return nxt, logits, inputs, caches, x
+
+
+def decode_step(pool, shape, weights: Dict, caches, token: int, pos: int):
+    """One greedy decode step of token `token` at position `pos` over the
+    per-layer caches (rows < pos filled; row pos written): (next id, logits)."""
+    x = oracle.embedding(torch.tensor([token], dtype=torch.int64), weights[("embed", -1)])
+    for l in range(shape.n_layers):
+        kc, vc = caches[l]
+        x = layer_prefill(pool, shape, layer_weights(weights, l), x, pos, kc, vc)
+    return head(pool, shape, weights[("final_norm", -1)], weights[("lm_head", -1)], x)

@@ -42,15 +42,30 @@ def assert_bf16_logits(got: torch.Tensor, ref: torch.Tensor, what: str = ""):
     return mx, cos
 
 
+# An operator fused into a linear's epilogue (RoPE on the q/k rows, SwiGLU over
+# the gate/up pair, the residual add): the linear's bf16 rounding of an fp32
+# (not fp64) sum may land one ulp away from the oracle's (2^-7 relative at
+# worst), and the fused operator rounds once more, from inputs that may carry
+# that ulp (RoPE mixes two of them): twice the single-operator bound.
+def assert_fused_close(got: torch.Tensor, ref: torch.Tensor, what: str = ""):
+    assert_close(got, ref, 2 * RTOL[ref.dtype], what)
+
+
 # A whole decoder layer is a chain of about twelve operators, each rounding
-# its output to bf16.  The per-operator bound (1e-2 of max(|ref|, rms(ref)),
-# just above one bf16 ulp, 2^-7) holds for every kernel on its own; at a
-# layer's output two 1-ulp differences can stack (a flipped rounding inside
-# the MLP carried into the final residual add, which rounds again), so the
-# layer bound is two ulps elementwise (2e-2) and 1e-2 in norm
-# (||gpu - ref|| <= 1e-2 ||ref||).
+# its output to bf16.  In norm the layer is held to 1e-2 (||gpu - ref|| <=
+# 1e-2 ||ref||: the ~1e-2 relative per-layer guidance of the Day-0 tutorial's
+# bisection step).  Elementwise, 1-ulp differences of the operators stack and
+# the tail grows with the number of elements compared: the oracle itself,
+# accumulating its linears and attention in fp32 instead of fp64, moves the
+# first layer's output on the 128-token prompt by 1.71e-2 of max(|ref|,
+# rms(ref)) at its worst element (relative norm 3.0e-3; `python -m
+# oracle.drift layer --tokens 128 --layer 0`).  A GPU path accumulating in
+# fp32 is held to twice that drift elementwise.
+LAYER_ELEMENTWISE = 3.5e-2
+
+
 def assert_layer_close(got: torch.Tensor, ref: torch.Tensor, what: str = ""):
-    assert_close(got, ref, 2e-2, what)
+    assert_close(got, ref, LAYER_ELEMENTWISE, what)
     g = got.detach().double().cpu()
     r = ref.detach().double().cpu()
     nrm = float((g - r).norm() / r.norm().clamp_min(1e-30))
