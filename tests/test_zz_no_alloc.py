@@ -5,14 +5,16 @@ Some callers cannot let a library allocate device memory while they call it
 wait on the allocator, code recording a CUDA graph under a capture mode that
 refuses allocation).  This variant keeps its partials in a fixed array of the
 library's device memory.  Checked here through the C ABI against the regular
-q2_argmax: identical indices and values (bit-exact, the argmax tolerance of
-these tests), on two calls in a row that share that array.  The file runs
-last so that a stop-at-first-failure run has already run everything else.
+q2_argmax and against the CPU oracle's argmax (first index of the maximum):
+identical indices and values (bit-exact, the argmax tolerance of these
+tests), on two calls in a row that share that array.  The file runs last so
+that a stop-at-first-failure run has already run everything else.
 """
 
 import pytest
 import torch
 
+import oracle
 import qwen2_decode_step_b200 as q2
 from synth import normal
 from tol import bits_equal
@@ -21,7 +23,7 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("dt,rows,n", [("f32", 64, 151936), ("bf16", 3, 4097), ("f32", 1, 1)])
-def test_noalloc_argmax_matches_argmax_on_two_calls_in_a_row(cuda_ok, dt, rows, n):
+def test_noalloc_argmax_matches_argmax_and_the_oracle_on_two_calls_in_a_row(cuda_ok, dt, rows, n):
     tdt = torch.float32 if dt == "f32" else torch.bfloat16
     for call in range(2):
         x = normal((rows, n), 1.0, 500 + call, dt).cuda()
@@ -36,6 +38,9 @@ def test_noalloc_argmax_matches_argmax_on_two_calls_in_a_row(cuda_ok, dt, rows, 
         torch.cuda.synchronize()
         assert torch.equal(got_i.cpu(), ref_i.cpu()), call
         assert bits_equal(got_v, ref_v), call
+        o_i, o_v = oracle.argmax(x.cpu())
+        assert torch.equal(got_i.cpu(), o_i), call
+        assert bits_equal(got_v, o_v), call
         if call == 1 and n > 10:
             assert int(got_i[0]) == 3
 
