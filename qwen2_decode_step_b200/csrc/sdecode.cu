@@ -16,13 +16,21 @@ using bf16 = __nv_bfloat16;
 
 namespace {
 
-constexpr int kCW = 8;                 // consumer warps
+constexpr int kCW = 8;                 // consumer warps (two warpgroups)
 constexpr int kCT = kCW * 32;          // consumer threads
-constexpr int kThreads = kCT + 32;     // + the producer warp
+constexpr int kThreads = kCT + 128;    // + the producer warpgroup (one warp of it streams)
+// Registers: the block is launched with kLaunchRegs per thread (what 384
+// threads and one block per SM allow: the register file of an SM sub-partition
+// holds three warps at 168); the producer warpgroup hands most of its share to
+// the consumer warpgroups.  The shares add up to the launch's total exactly.
+constexpr int kLaunchRegs = 168;
+constexpr int kProducerRegs = 56;
+constexpr int kConsumerRegs = 224;
+static_assert(kProducerRegs * 128 + kConsumerRegs * kCT == kLaunchRegs * kThreads,
+              "the warpgroups' register shares must add up to the launch's");
 constexpr int kSB = 24576;             // weight ring slot: 8 rows of K = 1536, or one down row
 constexpr int kAT = 64;                // attention keys per tile
 constexpr int kHD = 128;               // head dim of this kernel
-constexpr int kHalf = kHD / 2;
 constexpr int kTile = kAT * kHD * 2;   // one K (or V) tile
 constexpr int kAGMax = 8;              // query heads per kv head
 constexpr int kYMax = 256;             // rows per CTA of a short-row phase (parked row results)
@@ -38,47 +46,38 @@ enum { PH_QKV = 0, PH_ATTN = 1, PH_O = 2, PH_GU = 3, PH_DOWN = 4, PH_HEAD = 5 };
 __host__ __device__ inline size_t up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Shared-memory map (offsets from a 1024-byte aligned base: the attention
-// tiles are 128-byte-swizzled TMA boxes).
+// tiles are 128-byte-swizzled TMA boxes).  Every area but the weight ring and
+// the layer table has a fixed size and sits at a compile-time offset; the ring
+// (its depth is a launch parameter) and the layer table follow them.
+namespace sl {
+constexpr size_t kTiles = 0;  // [2 stages][K | V] tiles; the per-warp attention partials between items
+constexpr size_t kYrow = kTiles + 4 * (size_t)kTile;           // [kYMax] row results of a short-row phase
+constexpr size_t kPart = kYrow + (size_t)kYMax * 4;            // [kCW][kDMax] down-row column-slice sums
+constexpr size_t kXres = kPart + (size_t)kCW * kDMax * 4;       // [kDMax] this CTA's residual rows
+constexpr size_t kEbias = kXres + (size_t)kDMax * 4;           // [kQMax] q/k/v bias of this CTA's rows
+constexpr size_t kEcs = kEbias + (size_t)kQMax * 4;            // [kQMax / 2] RoPE (cos, sin) per row pair
+constexpr size_t kMlw = kEcs + (size_t)kQMax / 2 * 8;          // [kCW][kAGMax][2] per-warp attention max, sum
+constexpr size_t kAmv = kMlw + (size_t)kCW * kAGMax * 2 * 4;   // [kCW] per-warp argmax values
+constexpr size_t kAmi = kAmv + (size_t)kCW * 8;                // [kCW] per-warp argmax indices (8-aligned)
+constexpr size_t kXbuf = kAmi + (size_t)kCW * 8;               // [kHMax] bf16: the phase's input vector
+constexpr size_t kQst = kXbuf + (size_t)kHMax * 2;             // [kAGMax][kHD] bf16: one kv head's query heads
+constexpr size_t kKvn = kQst + (size_t)kAGMax * kHD * 2;       // [2][kHD] bf16: its new K and V rows
+constexpr size_t kAbar = kKvn + 2 * (size_t)kHD * 2;           // abar[2]
+constexpr size_t kFlags = kAbar + 2 * 8;                       // [8] ints
+constexpr size_t kRing = (kFlags + 8 * 4 + 1023) / 1024 * 1024;  // [ring][kSB] weight ring
+static_assert(kAmi % 8 == 0 && kXbuf % 16 == 0 && kAbar % 8 == 0, "shared-memory alignment");
+}  // namespace sl
+
 struct SLay {
-  size_t tiles, ring, layers, yrow, part, xres, ebias, ecs, mlw, amv, ami, xbuf, qst, kvn, bars, flags, total;
+  size_t ring, bars, layers, total;
 };
 
 __host__ __device__ inline SLay slayout(int ring, int L) {
   SLay Y;
-  size_t o = 0;
-  Y.tiles = o;  // [2 stages][K | V] tiles; the per-warp attention partials between items
-  o += 4 * (size_t)kTile;
-  Y.ring = o;
-  o += (size_t)ring * kSB;
-  Y.layers = o;  // [L] layer weight pointers
-  o = up(o + (size_t)L * sizeof(PLayer), 16);
-  Y.yrow = o;  // [kYMax] row results of a short-row phase
-  o += (size_t)kYMax * 4;
-  Y.part = o;  // [kCW][kDMax] per-warp column-slice sums of the down rows
-  o += (size_t)kCW * kDMax * 4;
-  Y.xres = o;  // [kDMax] this CTA's rows of the residual stream
-  o += (size_t)kDMax * 4;
-  Y.ebias = o;  // [kQMax] q/k/v bias of this CTA's rows
-  o += (size_t)kQMax * 4;
-  Y.ecs = o;  // [kQMax / 2] RoPE (cos, sin) of this CTA's row pairs
-  o += (size_t)kQMax / 2 * 8;
-  Y.mlw = o;  // [kCW][kAGMax][2] per-warp attention max and sum
-  o += (size_t)kCW * kAGMax * 2 * 4;
-  Y.amv = o;  // [kCW] per-warp argmax values
-  o += kCW * 4;
-  Y.ami = up(o, 8);  // [kCW] per-warp argmax indices
-  o = Y.ami + kCW * 8;
-  Y.xbuf = up(o, 16);  // [kHMax] bf16: the phase's input vector
-  o = Y.xbuf + (size_t)kHMax * 2;
-  Y.qst = o;  // [kAGMax][kHD] bf16: one kv head's query heads
-  o += (size_t)kAGMax * kHD * 2;
-  Y.kvn = o;  // [2][kHD] bf16: the new K and V rows of that kv head
-  o += 2 * (size_t)kHD * 2;
-  Y.bars = up(o, 8);  // full[ring], empty[ring], abar[2]
-  o = Y.bars + (2 * (size_t)ring + 2) * 8;
-  Y.flags = o;
-  o += 8 * 4;
-  Y.total = o + 1024;  // slack for aligning the base
+  Y.ring = sl::kRing;
+  Y.bars = Y.ring + (size_t)ring * kSB;  // full[ring], empty[ring]
+  Y.layers = up(Y.bars + 2 * (size_t)ring * 8, 16);  // [L] layer weight pointers
+  Y.total = Y.layers + (size_t)L * sizeof(PLayer) + 1024;  // + slack for aligning the base
   return Y;
 }
 
@@ -145,21 +144,6 @@ struct Poll {
   __device__ bool stop(uint64_t t0) const {
     return *reinterpret_cast<volatile unsigned*>(gave_up) != 0u || gtimer() - t0 > deadline_ns;
   }
-  // one word
-  __device__ uint32_t get(const uint64_t* w, uint32_t tag) const {
-    uint64_t v;
-    asm volatile("ld.volatile.global.u64 %0, [%1];" : "=l"(v) : "l"(w) : "memory");
-    if ((uint32_t)(v >> 32) == tag) return (uint32_t)v;
-    const uint64_t t0 = gtimer();
-    for (unsigned it = 1;; ++it) {
-      asm volatile("ld.volatile.global.u64 %0, [%1];" : "=l"(v) : "l"(w) : "memory");
-      if ((uint32_t)(v >> 32) == tag) return (uint32_t)v;
-      if ((it & 15u) == 0 && stop(t0)) {
-        fail();
-        return (uint32_t)v;
-      }
-    }
-  }
   // two consecutive words (16-byte aligned)
   __device__ uint2 get2(const uint64_t* w, uint32_t tag) const {
     uint32_t d0, t0_, d1, t1_;
@@ -183,6 +167,39 @@ struct Poll {
   }
 };
 
+// Polls up to N 16-byte lines until both words of each carry `tag`: line i
+// (used where bit i of `mask` is set) is at base + (i / 2) * pair_stride +
+// (i odd ? off1 : off0) words.  Every outstanding load is issued before any is
+// checked, so the lines cost one round trip together rather than one each.
+template <int N>
+__device__ __forceinline__ void get_lines(const Poll& pl, const uint64_t* base, size_t pair_stride, size_t off0,
+                                          size_t off1, uint32_t mask, uint32_t tag, uint2 (&out)[N]) {
+  uint32_t pending = mask;
+  uint64_t t0 = 0;
+  for (unsigned it = 0; pending; ++it) {
+    uint4 v[N];
+#pragma unroll
+    for (int i = 0; i < N; ++i)
+      if ((pending >> i) & 1u)
+        asm volatile("ld.volatile.global.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(v[i].x), "=r"(v[i].y), "=r"(v[i].z), "=r"(v[i].w)
+                     : "l"(base + (size_t)(i >> 1) * pair_stride + ((i & 1) ? off1 : off0))
+                     : "memory");
+#pragma unroll
+    for (int i = 0; i < N; ++i)
+      if ((pending >> i) & 1u) {
+        out[i] = make_uint2(v[i].x, v[i].z);
+        if (v[i].y == tag && v[i].w == tag) pending &= ~(1u << i);
+      }
+    if (!pending) break;
+    if (it == 0) t0 = gtimer();
+    if ((it & 7u) == 7u && pl.stop(t0)) {
+      pl.fail();
+      break;
+    }
+  }
+}
+
 __device__ __forceinline__ uint32_t bf2_bits(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&v);
@@ -191,8 +208,6 @@ __device__ __forceinline__ uint32_t bf2_bits(bf16 lo, bf16 hi) {
   return (uint32_t)*reinterpret_cast<const uint16_t*>(&lo) |
          ((uint32_t)*reinterpret_cast<const uint16_t*>(&hi) << 16);
 }
-__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
 __device__ __forceinline__ float silu_mul(float gv, float uv) { return uv * (gv / (1.0f + expf(-gv))); }
 
@@ -301,24 +316,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int RING = p.ring;
   const int L = p.L;
   const SLay Y = slayout(RING, L);
-  uint8_t* tiles = smem + Y.tiles;
-  uint8_t* ring = smem + Y.ring;
+  uint8_t* tiles = smem + sl::kTiles;
+  uint8_t* ring = smem + sl::kRing;
   PLayer* layers = reinterpret_cast<PLayer*>(smem + Y.layers);
-  float* yrow = reinterpret_cast<float*>(smem + Y.yrow);
-  float* part = reinterpret_cast<float*>(smem + Y.part);
-  float* xres = reinterpret_cast<float*>(smem + Y.xres);
-  float* ebias = reinterpret_cast<float*>(smem + Y.ebias);
-  float2* ecs = reinterpret_cast<float2*>(smem + Y.ecs);
-  float* mlw = reinterpret_cast<float*>(smem + Y.mlw);
-  float* amv = reinterpret_cast<float*>(smem + Y.amv);
-  long long* ami = reinterpret_cast<long long*>(smem + Y.ami);
-  bf16* xbuf = reinterpret_cast<bf16*>(smem + Y.xbuf);
-  bf16* qst = reinterpret_cast<bf16*>(smem + Y.qst);
-  bf16* kvn = reinterpret_cast<bf16*>(smem + Y.kvn);
+  float* yrow = reinterpret_cast<float*>(smem + sl::kYrow);
+  float* part = reinterpret_cast<float*>(smem + sl::kPart);
+  float* xres = reinterpret_cast<float*>(smem + sl::kXres);
+  float* ebias = reinterpret_cast<float*>(smem + sl::kEbias);
+  float2* ecs = reinterpret_cast<float2*>(smem + sl::kEcs);
+  float* mlw = reinterpret_cast<float*>(smem + sl::kMlw);
+  float* amv = reinterpret_cast<float*>(smem + sl::kAmv);
+  long long* ami = reinterpret_cast<long long*>(smem + sl::kAmi);
+  bf16* xbuf = reinterpret_cast<bf16*>(smem + sl::kXbuf);
+  bf16* qst = reinterpret_cast<bf16*>(smem + sl::kQst);
+  bf16* kvn = reinterpret_cast<bf16*>(smem + sl::kKvn);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Y.bars);
   uint64_t* empty = full + RING;
-  uint64_t* abar = empty + RING;
-  int* s_flags = reinterpret_cast<int*>(smem + Y.flags);  // [0] position, [1] step, [2] tiles pre-issued
+  uint64_t* abar = reinterpret_cast<uint64_t*>(smem + sl::kAbar);
+  int* s_flags = reinterpret_cast<int*>(smem + sl::kFlags);  // [0] position, [1] step, [2] tiles pre-issued
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x, bid = blockIdx.x;
@@ -354,8 +369,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   // One lane walks this CTA's stages of the whole step and issues one bulk
   // copy per stage as soon as its slot is free; a second cursor runs
   // l2_ahead stages in front and pulls them into L2.
-  if (warp == kCW) {
-    if (lane == 0) {
+  if (warp >= kCW) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
+    if (warp == kCW && lane == 0) {
       const uint64_t pol = policy_evict_first();
       Cursor cur, ahead;
       cur.start(p, layers, bid, G, nph);
@@ -397,6 +413,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // =============================================================== consumers
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kConsumerRegs));
   const int ct = tid;
   const int Gq = p.nh / p.nkv;
   const int half = p.hd >> 1;
@@ -428,7 +445,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
   // the phase's input vector into xbuf: from tagged words (bf16 pairs) ...
   auto stage_tagged = [&](const uint64_t* ll, int nwords, uint32_t tag) {
-    for (int v = ct; v < nwords / 2; v += kCT) reinterpret_cast<uint2*>(xbuf)[v] = pl.get2(ll + 2 * v, tag);
+    uint2 got[2];
+    uint32_t mask = 0;
+#pragma unroll
+    for (int k = 0; k < 2; ++k)
+      if (ct + kCT * k < nwords / 2) mask |= 1u << k;
+    get_lines<2>(pl, ll, 0, 2 * (size_t)ct, 2 * (size_t)(ct + kCT), mask, tag, got);
+#pragma unroll
+    for (int k = 0; k < 2; ++k)
+      if ((mask >> k) & 1u) reinterpret_cast<uint2*>(xbuf)[ct + kCT * k] = got[k];
     csync();
   };
   // ... or from plain bf16 memory
@@ -500,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // The stages of the down phase: one row per stage, warp w takes column
   // pieces [w * cpw, (w + 1) * cpw) of it.
-  auto consume_long = [&](const PW& pw, const float (&xs)[NQ][8]) {
+  auto consume_long = [&](const PW& pw, const uint4 (&xs)[NQ]) {
     const int cpw = pw.K / 8 / kCW;
     for (int r = pw.r0; r < pw.r1; r += pw.rs, ++gs) {
       const int slot = c_slot;
@@ -515,10 +540,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int q = 0; q < NQ; ++q) {
         if (lane + 32 * q < cpw) {
-          float wf[8];
+          float wf[8], xf[8];
           unpack16<bf16>(wrow[lane + 32 * q], wf);
+          unpack16<bf16>(xs[q], xf);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) a[e & 3] = fmaf(wf[e], xs[q][e], a[e & 3]);
+          for (int e = 0; e < 8; ++e) a[e & 3] = fmaf(wf[e], xf[e], a[e & 3]);
         }
       }
       const float y = warp_sum((a[0] + a[1]) + (a[2] + a[3]));
@@ -559,6 +585,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   };
   const int aitems = p.nkv * p.nsplit;
+  // The first two tiles of this CTA's first attention item of layer l, issued
+  // a layer ahead (at the start for layer 0, else when layer l - 1's
+  // attention is done with the buffers) so that they land behind the weight
+  // copies queued on this SM long before they are needed; the tile holding
+  // the new position gets that row patched in later.
+  auto prefetch_tiles = [&](int l) {
+    if (ct != 0) return;
+    s_flags[2] = 0;
+    if (bid < aitems && l < L) {
+      const AItem a = attn_item(bid);
+      for (int q = 0; q < 2 && a.t0 + q < a.t1; ++q) {
+        tile_issue(l, a.gq, a.t0 + q, ac + q);
+        s_flags[2] = q + 1;
+      }
+    }
+  };
+  prefetch_tiles(0);
 
   for (int ph = 0; ph < nph; ++ph) {
     const int kind = phase_kind(L, ph);
@@ -580,18 +623,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         if ((i & 1) == 0 && n / p.hd < p.nh + p.nkv)
           ecs[i >> 1] = __ldg(p.rope + (size_t)pos * half + ((n % p.hd) >> 1));
       }
-      // the first two tiles of this CTA's first attention item of the layer
-      // (the tile holding the new position gets that row patched in later)
-      if (ct == 0) {
-        s_flags[2] = 0;
-        if (bid < aitems) {
-          const AItem a = attn_item(bid);
-          for (int q = 0; q < 2 && a.t0 + q < a.t1; ++q) {
-            tile_issue(l, a.gq, a.t0 + q, ac + q);
-            s_flags[2] = q + 1;
-          }
-        }
-      }
     } else if (kind == PH_GU) {
       load_nw(layers[l].post_norm, nwr);
     } else if (kind == PH_HEAD) {
@@ -612,7 +643,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int mi = lane >> 3, mr = lane & 7;  // ldmatrix: lane addresses row mr of matrix mi
       const float sl2 = p.scale * kLog2e;
       const uint32_t tq = rtag(ph - 1), ta = wtag(ph);
-      if (ctr && ct == 0) ctr[1] = gtimer();
       for (int item = bid; item < aitems; item += G) {
         const AItem a = attn_item(item);
         if (a.t0 >= a.t1) continue;
@@ -640,6 +670,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           r[j + 1 + half] = __ushort_as_bfloat16((unsigned short)(d.y >> 16));
         }
         csync();
+        if (ctr && ct == 0 && item == bid) ctr[1] = gtimer();  // attention: q and the new K/V row in
         // A fragments of the query heads (bf16, unscaled); rows fr >= Gq are zero
         uint32_t qa[8][2];
 #pragma unroll
@@ -670,17 +701,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const uint32_t kt = smem_u32(tk);
           const uint32_t vt = kt + (uint32_t)kTile;
-          // ---- scores of this warp's 16 keys: s0 keys +0..7, s1 keys +8..15
+          // ---- scores of this warp's 16 keys: s0 keys +0..7, s1 keys +8..15, each
+          // summed over the head dims in two independent chains (even and odd
+          // k-steps) to halve the dependent MMA latency
           float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
           {
+            float s0b[4] = {0.f, 0.f, 0.f, 0.f}, s1b[4] = {0.f, 0.f, 0.f, 0.f};
             const int key = wq * 16 + ((mi >> 1) << 3) + mr;
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
               const int dim = 16 * kk + ((mi & 1) << 3);
               uint32_t r0, r1, r2, r3;
               ldsm_x4(kt + (uint32_t)((dim >> 6) * 8192) + swz_off(key, dim & 63), r0, r1, r2, r3);
-              mma16816(s0, qa[kk][0], qa[kk][1], r0, r1);
-              mma16816(s1, qa[kk][0], qa[kk][1], r2, r3);
+              mma16816((kk & 1) ? s0b : s0, qa[kk][0], qa[kk][1], r0, r1);
+              mma16816((kk & 1) ? s1b : s1, qa[kk][0], qa[kk][1], r2, r3);
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              s0[e] += s0b[e];
+              s1[e] += s1b[e];
             }
           }
           // ---- online softmax for head fr over keys kb + 2fc, +1 and kb + 8 + 2fc, +1
@@ -746,6 +785,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (ct == 0 && i + 2 < nt) tile_issue(l, a.gq, t + 2, li + 2);
         }
         ac += nt;
+        if (ctr && ct == 0 && item == bid) ctr[2] = gtimer();  // attention: tiles done
 
         // ---- the four warps of each group (max, sum, unnormalised output),
         // merged; the tile buffers are free now (every tile of the item was
@@ -764,62 +804,118 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         csync();
-        // thread i takes dims (2 dp, 2 dp + 1) of head hh
-        for (int i = ct; i < Gq * half; i += kCT) {
-          const int hh = i / half, dp = i % half, d = 2 * dp, w0 = 4 * (d >> 6);
+        // thread ct takes dims (2 dp, 2 dp + 1) of head hh for items i = ct, ct + kCT
+        // (Gq * half <= 2 kCT): this split's (max, sum, output) of them
+        float cM[2], cL[2], cO0[2], cO1[2];
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int i = ct + kCT * k;
+          cM[k] = -INFINITY;
+          cL[k] = cO0[k] = cO1[k] = 0.f;
+          if (i >= Gq * half) continue;
+          const int hh = i / half, d = 2 * (i % half), w0 = 4 * (d >> 6);
           float M = -INFINITY;
 #pragma unroll
           for (int w = w0; w < w0 + 4; ++w) M = fmaxf(M, mlw[(w * kAGMax + hh) * 2]);
           const float Ms = M == -INFINITY ? 0.f : M;
-          float O0 = 0.f, O1 = 0.f, Ls = 0.f;
 #pragma unroll
           for (int w = w0; w < w0 + 4; ++w) {
             const float e = exp2f(mlw[(w * kAGMax + hh) * 2] - Ms);
             const float* ow = Ow + ((size_t)w * kAGMax + hh) * 64 + (d & 63);
-            O0 = fmaf(e, ow[0], O0);
-            O1 = fmaf(e, ow[1], O1);
-            Ls = fmaf(e, mlw[(w * kAGMax + hh) * 2 + 1], Ls);
+            cO0[k] = fmaf(e, ow[0], cO0[k]);
+            cO1[k] = fmaf(e, ow[1], cO1[k]);
+            cL[k] = fmaf(e, mlw[(w * kAGMax + hh) * 2 + 1], cL[k]);
           }
-          uint64_t* pbase = p.ll.part + ((size_t)(a.gq * kSplitMax + a.split) * Gq + hh) * (kHD + 2);
-          if (a.split > 0) {  // a partial for the first split of this kv head
-            ll_put2(pbase + d, __float_as_uint(O0), __float_as_uint(O1), ta);
-            if (dp == 0) ll_put2(pbase + kHD, __float_as_uint(M), __float_as_uint(Ls), ta);
-          } else {
-            // the first split merges the others in split order:
-            // o = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s
-            for (int sp = 1; sp < a.nact; ++sp) {
-              const uint64_t* ob = p.ll.part + ((size_t)(a.gq * kSplitMax + sp) * Gq + hh) * (kHD + 2);
-              const uint2 ml = pl.get2(ob + kHD, rtag(ph));
-              const uint2 ov = pl.get2(ob + d, rtag(ph));
-              const float ms = __uint_as_float(ml.x), lsp = __uint_as_float(ml.y);
-              const float Mn = fmaxf(M, ms);
-              const float ea = exp2f(M - Mn), eb = exp2f(ms - Mn);
-              O0 = O0 * ea + __uint_as_float(ov.x) * eb;
-              O1 = O1 * ea + __uint_as_float(ov.y) * eb;
-              Ls = Ls * ea + lsp * eb;
-              M = Mn;
+          cM[k] = M;
+        }
+        const size_t hstride = kHD + 2;  // words per (split, head)
+        if (a.split > 0) {  // a partial for the first split of this kv head
+          uint64_t* pb = p.ll.part + (size_t)(a.gq * kSplitMax + a.split) * Gq * hstride;
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const int i = ct + kCT * k;
+            if (i >= Gq * half) continue;
+            const int hh = i / half, d = 2 * (i % half);
+            ll_put2(pb + hh * hstride + d, __float_as_uint(cO0[k]), __float_as_uint(cO1[k]), ta);
+            if (d == 0) ll_put2(pb + hh * hstride + kHD, __float_as_uint(cM[k]), __float_as_uint(cL[k]), ta);
+          }
+        } else {
+          // The first split merges the others in split order:
+          // o = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s.  Their partials
+          // are staged into the (free) tile buffer a chunk of splits at a
+          // time, each thread polling its share of the chunk's lines at once.
+          const int chunk = (int)(4 * (size_t)kTile / (Gq * hstride * 4));  // splits that fit the buffer
+          float* pst = reinterpret_cast<float*>(tiles);
+          const uint64_t* pb0 = p.ll.part + (size_t)(a.gq * kSplitMax) * Gq * hstride;
+          for (int s0 = 1; s0 < a.nact; s0 += chunk) {
+            const int ns = min(chunk, a.nact - s0);
+            const int nlines = ns * Gq * (int)hstride / 2;
+            csync();  // the buffer's previous contents (partials, earlier chunk) are read
+            for (int l0 = 0; l0 < nlines; l0 += 4 * kCT) {
+              uint2 got[4];
+              uint32_t mask = 0;
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                if (l0 + ct + kCT * k < nlines) mask |= 1u << k;
+              get_lines<4>(pl, pb0 + (size_t)s0 * Gq * hstride + 2 * (size_t)l0, 2 * 2 * kCT, 2 * (size_t)ct,
+                           2 * (size_t)(ct + kCT), mask, rtag(ph), got);
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                if ((mask >> k) & 1u)
+                  reinterpret_cast<uint2*>(pst)[l0 + ct + kCT * k] =
+                      make_uint2(got[k].x, got[k].y);
             }
-            const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
-            ll_put(p.ll.att + (size_t)(a.gq * Gq + hh) * half + dp, bf2_bits(O0 * inv, O1 * inv), ta);
+            csync();
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+              const int i = ct + kCT * k;
+              if (i >= Gq * half) continue;
+              const int hh = i / half, d = 2 * (i % half);
+              for (int sp = 0; sp < ns; ++sp) {
+                const float* ps = pst + ((size_t)sp * Gq + hh) * hstride;
+                const float ms = ps[kHD], lsp = ps[kHD + 1];
+                const float Mn = fmaxf(cM[k], ms);
+                const float ea = exp2f(cM[k] - Mn), eb = exp2f(ms - Mn);
+                cO0[k] = cO0[k] * ea + ps[d] * eb;
+                cO1[k] = cO1[k] * ea + ps[d + 1] * eb;
+                cL[k] = cL[k] * ea + lsp * eb;
+                cM[k] = Mn;
+              }
+            }
+          }
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const int i = ct + kCT * k;
+            if (i >= Gq * half) continue;
+            const int hh = i / half, dp = i % half;
+            const float inv = cL[k] > 0.f ? 1.f / cL[k] : 0.f;
+            ll_put(p.ll.att + (size_t)(a.gq * Gq + hh) * half + dp, bf2_bits(cO0[k] * inv, cO1[k] * inv), ta);
           }
         }
         fence_proxy_async_smem();  // the tile buffer is a TMA destination again later
         csync();
       }
+      prefetch_tiles(l + 1);
     } else if (kind == PH_DOWN) {
-      float xs[NQ][8];  // this lane's pieces of the warp's column slice of s
+      uint4 xs[NQ];  // this lane's pieces of the warp's column slice of s (bf16)
       const int cpw = pw.K / 8 / kCW;
-      const uint32_t tg = rtag(ph - 1);
+      {
+        const uint64_t* sbase = p.ll.s + (size_t)(warp * cpw + lane) * 4;
+        constexpr int QH = (NQ + 1) / 2;  // pieces polled per batch
 #pragma unroll
-      for (int q = 0; q < NQ; ++q) {
-        const int c = lane + 32 * q;
-        if (c < cpw) {
-          const uint64_t* w = p.ll.s + (size_t)(warp * cpw + c) * 4;
-          const uint2 a = pl.get2(w, tg), b = pl.get2(w + 2, tg);
-          unpack16<bf16>(make_uint4(a.x, a.y, b.x, b.y), xs[q]);
-        } else {
+        for (int q0 = 0; q0 < NQ; q0 += QH) {
+          uint2 got[2 * QH];
+          uint32_t mask = 0;
 #pragma unroll
-          for (int e = 0; e < 8; ++e) xs[q][e] = 0.f;
+          for (int q = 0; q < QH; ++q)
+            if (q0 + q < NQ && lane + 32 * (q0 + q) < cpw) mask |= 3u << (2 * q);
+          get_lines<2 * QH>(pl, sbase + (size_t)(32 * q0) * 4, 32 * 4, 0, 2, mask, rtag(ph - 1), got);
+#pragma unroll
+          for (int q = 0; q < QH; ++q)
+            if (q0 + q < NQ)
+              xs[q0 + q] = (mask >> (2 * q)) & 1u
+                               ? make_uint4(got[2 * q].x, got[2 * q].y, got[2 * q + 1].x, got[2 * q + 1].y)
+                               : make_uint4(0u, 0u, 0u, 0u);
         }
       }
       if (ctr && ct == 0) ctr[1] = gtimer();
@@ -850,7 +946,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---- phase epilogue from the parked row results and staged operands
     csync();
-    if (ctr && ct == 0) ctr[2] = gtimer();
+    if (ctr && ct == 0 && kind != PH_ATTN) ctr[2] = gtimer();
     const uint32_t tw = wtag(ph);
     if (kind == PH_QKV) {
       const size_t loff = (size_t)l * p.kv_layer_stride;
@@ -1066,6 +1162,15 @@ q2_status launch_sdecode(const SDecode& p, const CUtensorMap& kmap, const CUtens
     return Q2_ERR_SHAPE;
   }
   auto kern = sdecode_kernel<kNCH, kNQ>;
+  // The warpgroups' register split assumes exactly kLaunchRegs per thread at
+  // launch; with any other count the split could not be honoured.
+  cudaFuncAttributes fa;
+  Q2_CUDA_TRY(cudaFuncGetAttributes(&fa, kern));
+  if (fa.numRegs != kLaunchRegs) {
+    set_error("streaming decode: the kernel was built with " + std::to_string(fa.numRegs) +
+              " registers per thread, its register split assumes " + std::to_string(kLaunchRegs));
+    return Q2_ERR_CUDA;
+  }
   Q2_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Y.total));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(G);
