@@ -9,6 +9,9 @@
 // Definition followed: the attention sketch of the Day-0 adaptation tutorial
 // (step 5): scores = q k^T * scale, causal mask, stable softmax, times V; the
 // LLAISYS final report (section 3.2) computes attention scores in float.
+#include <cstdlib>
+#include <string>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -233,6 +236,16 @@ __global__ void attn_combine_kernel(AttnRows a, int nsplit, const float* part_o,
   out[d] = from_f<T>(den > 0.f ? o / den : 0.f);
 }
 
+// Prefill attention implementation: 0 the tcgen05 kernel (default), 1 the
+// mma.sync kernel (Q2_PREFILL_ATTN=mma selects it, for comparisons).
+int prefill_attn_impl() {
+  static const int v = [] {
+    const char* e = getenv("Q2_PREFILL_ATTN");
+    return (e && std::string(e) == "mma") ? 1 : 0;
+  }();
+  return v;
+}
+
 int attn_splits(int rows, int nkv, int max_keys) {
   long long ctas = (long long)rows * nkv;
   // as many splits as fit one wave of two CTAs per SM (a partial second wave
@@ -271,7 +284,15 @@ static q2_status attn_t(const AttnRows& a, int nsplit, void* scratch, cudaStream
 }
 
 q2_status launch_attention(const AttnRows& a, int nsplit, void* scratch, int dtype,
-                           cudaStream_t st, bool pdl) {
+                           cudaStream_t st, bool pdl, int* err) {
+  if (attn_tc_supported(a, dtype) && prefill_attn_impl() == 0) {
+    int* e = err ? err : op_error_flag();
+    if (!e) {
+      set_error("attention: no error word");
+      return Q2_ERR_CUDA;
+    }
+    return launch_attn_tc(a, e, st);
+  }
   if (attn_prefill_mma_supported(a, dtype)) return launch_attn_prefill_mma(a, st, pdl);
   if (a.rows == 0) return Q2_OK;
   if (a.nkv <= 0 || a.nh % a.nkv != 0 || a.nh / a.nkv > kGMax) {

@@ -1,0 +1,447 @@
+// attn_tc.cu -- causal GQA attention of a block of query rows of one sequence
+// (prefill) on the sm_100a tensor cores: tcgen05.mma with the score and
+// output accumulators in tensor memory, operands in 128-byte-swizzled shared
+// memory, K/V tiles by TMA.
+//
+// One CTA per (128 query rows, query head); 256 threads:
+//   warp 0     TMA: the Q block once (two 64-dim boxes), then K and V tiles
+//              of 128 keys into a two-stage ring
+//   warp 1     allocates tensor memory; one thread issues the MMAs:
+//                S_j  = Q K_j^T   M = 128 rows, N = 128 keys, K = 128 dims,
+//                                 into TMEM S[j % 2] (fp32)
+//                O   += P_j V_j   M = 128 rows, N = 128 dims, K = 128 keys,
+//                                 into TMEM O (fp32), once with P's bf16 high
+//                                 part and once with its low part (P keeps
+//                                 ~16 significant bits); V is the MN-major
+//                                 operand (dims contiguous, as the cache
+//                                 stores it)
+//              in the order S_0, S_1, O += P_0 V_0, S_2, O += P_1 V_1, ...,
+//              so a tile's scores are computed while the softmax of the tile
+//              before runs
+//   warps 4-7  softmax: thread r owns query row r (TMEM lane r).  It reads its
+//              row of S_j, applies the scale and the causal mask, keeps the
+//              running max m and sum l (O is rescaled only when the max grows
+//              by more than 2^8, so most tiles leave O untouched), writes
+//              P_j = 2^(s - m) as bf16(P) and bf16(P - bf16(P)) into shared
+//              memory as the A operands of the P V products, and at the end
+//              writes O / l in bf16.
+// Every wait is bounded by a deadline; one that runs out sets value 2 in the
+// caller's error word and the kernel carries on to its end.
+//
+// Definition followed: the attention of the Day-0 adaptation tutorial (step
+// 5): scores q k^T * scale, causal mask (query i of a block at positions
+// pos0.. sees keys j <= pos0 + i), stable softmax, times V; query head h reads
+// kv head h / (nh / nkv).
+#include "common.cuh"
+#include "kernels.h"
+#include "tma.h"
+
+namespace q2 {
+
+using bf16 = __nv_bfloat16;
+
+namespace {
+
+constexpr int kQB = 128;   // query rows per CTA (MMA M)
+constexpr int kKB = 128;   // keys per tile
+constexpr int kHD = 128;   // head dim
+constexpr int kThreads = 256;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescale = 8.0f;  // O is rescaled when the running max grows by more than this (log2)
+constexpr uint64_t kDeadlineNs = 2000ull * 1000 * 1000;
+
+constexpr size_t kBox = (size_t)128 * 64 * 2;  // one 128-row x 64-column bf16 box: 16 KB
+constexpr size_t kQOff = 0;                    // Q: 2 boxes
+constexpr size_t kKVOff = 2 * kBox;            // [2 stages][K: 2 boxes | V: 2 boxes]
+constexpr size_t kStage = 4 * kBox;
+constexpr size_t kPOff = kKVOff + 2 * kStage;  // P high: 2 boxes of 128 rows x 64 keys, then P low
+constexpr size_t kBarOff = kPOff + 2 * 2 * kBox;
+constexpr size_t kSmem = kBarOff + 16 * 8 + 16 + 1024;  // barriers, TMEM base, alignment slack
+
+__device__ __forceinline__ uint64_t gtimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = gtimer();
+  for (;;) {
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (gtimer() - t0 > kDeadlineNs) return false;
+  }
+}
+
+// Shared-memory descriptor of a K-major, 128-byte-swizzled operand tile whose
+// 8-row groups are 1024 bytes apart (a TMA box of 64 bf16 columns with
+// 128-byte swizzle): start >> 4, leading offset 16 B (unused), stride offset
+// 1024 B, descriptor version 1, swizzle mode 2 (128 B).
+__device__ __forceinline__ uint64_t desc_kmajor(uint32_t saddr) {
+  return ((uint64_t)((saddr >> 4) & 0x3FFFu)) | (1ull << 16) | ((uint64_t)(1024 >> 4) << 32) | (1ull << 46) |
+         (2ull << 61);
+}
+
+// Descriptor of an MN-major, 128-byte-swizzled operand: the MN dimension
+// contiguous (64 elements = one 128-byte row of a swizzle atom), the K
+// dimension along the rows (8 rows = one 1024-byte atom).  Leading offset:
+// bytes between 64-element MN blocks (the next TMA box); stride offset: bytes
+// between 8-row K groups (1024).
+__device__ __forceinline__ uint64_t desc_mnmajor(uint32_t saddr, uint32_t mn_block_bytes) {
+  return ((uint64_t)((saddr >> 4) & 0x3FFFu)) | ((uint64_t)((mn_block_bytes >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)(1024 >> 4) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, A K-major,
+// B K-major (b_mn = 0) or MN-major (b_mn = 1), N = n, M = 128.
+__host__ __device__ constexpr uint32_t idesc(int n, int b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)b_mn << 16) | ((uint32_t)(n >> 3) << 17) |
+         ((uint32_t)(kQB >> 4) << 24);
+}
+
+__device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void mma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(id), "r"(acc)
+      : "memory");
+}
+
+__device__ __forceinline__ void commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+// 32 consecutive fp32 columns of this thread's TMEM lane (no wait).
+__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
+      "%13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, "
+      "%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+        "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+        "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
+      "%13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, "
+      "%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+struct AttnTc {
+  int rows;        // query rows of the chunk
+  int nh, nkv;     // heads
+  int pos0;        // position of query row 0 (row i sees keys 0 .. pos0 + i)
+  int kv_x_step;   // K/V tensor maps: the tile origin of kv head g is at
+  int kv_y_step;   // (x, y) = (g * kv_x_step, g * kv_y_step + first key)
+  float scale;
+  void* out;
+  long long out_row_stride;  // elements
+  int* err;
+};
+
+}  // namespace
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                   const __grid_constant__ CUtensorMap tv, const AttnTc a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarOff);
+  uint64_t* q_full = bars + 0;
+  uint64_t* kv_full = bars + 1;   // [2]
+  uint64_t* kv_empty = bars + 3;  // [2]
+  uint64_t* s_full = bars + 5;    // [2]
+  uint64_t* p_full = bars + 7;    // [2]
+  uint64_t* o_done = bars + 9;
+  uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(bars + 16);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ntq = (a.rows + kQB - 1) / kQB;
+  const int qt = ntq - 1 - (int)blockIdx.x;  // the longest (last) row blocks first
+  const int h = blockIdx.y, kvh = h / (a.nh / a.nkv);
+  const int q0 = qt * kQB;
+  const int last_row = min(q0 + kQB, a.rows) - 1;
+  const int nkt = (a.pos0 + last_row) / kKB + 1;  // key tiles up to the block's last visible key
+  const int keys_end = a.pos0 + a.rows;            // keys written so far (later rows are stale)
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 128);
+    }
+    mbar_init(o_done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {  // S[0], S[1], O: 3 x 128 fp32 columns (allocated as 512)
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_base_s)),
+                 "r"(512)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_base_s);
+  const uint32_t tS0 = tmem, tO = tmem + 256;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA
+    if (lane == 0) {
+      mbar_arrive_expect_tx(q_full, 2 * kBox);
+      for (int b = 0; b < 2; ++b) tma_load_2d(smem + kQOff + b * kBox, &tq, h * kHD + 64 * b, q0, q_full);
+      const int xbase = kvh * a.kv_x_step, ybase = kvh * a.kv_y_step;
+      for (int j = 0; j < nkt; ++j) {
+        const int s = j & 1;
+        if (j >= 2 && !wait_bar(&kv_empty[s], (uint32_t)(((j >> 1) - 1) & 1))) atomicOr(a.err, 2);
+        uint8_t* st = smem + kKVOff + s * kStage;
+        mbar_arrive_expect_tx(&kv_full[s], 4 * kBox);
+        for (int b = 0; b < 2; ++b) {
+          tma_load_2d(st + b * kBox, &tk, xbase + 64 * b, ybase + j * kKB, &kv_full[s]);
+          tma_load_2d(st + (2 + b) * kBox, &tv, xbase + 64 * b, ybase + j * kKB, &kv_full[s]);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA
+    if (lane == 0) {
+      constexpr uint32_t id_s = idesc(kKB, 0);  // S = Q K^T: both K-major (dims contiguous)
+      constexpr uint32_t id_o = idesc(kHD, 1);  // O += P V: P K-major (keys contiguous), V MN-major
+      const uint32_t qa = smem_u32(smem + kQOff);
+      if (!wait_bar(q_full, 0)) atomicOr(a.err, 2);
+      auto pv = [&](int j) {  // O += P_j V_j
+        const int s = j & 1;
+        if (!wait_bar(&p_full[s], (uint32_t)((j >> 1) & 1))) atomicOr(a.err, 2);
+        fence_after();
+        const uint32_t pa = smem_u32(smem + kPOff);
+        const uint32_t va = smem_u32(smem + kKVOff + (size_t)s * kStage + 2 * kBox);
+#pragma unroll
+        for (int k = 0; k < kKB / 16; ++k) {  // 16 keys per MMA
+          const uint32_t poff = (uint32_t)((k >> 2) * kBox) + (uint32_t)((k & 3) * 32);
+          const uint64_t db = desc_mnmajor(va + (uint32_t)(k * 16 * 128), (uint32_t)kBox);
+          mma(tO, desc_kmajor(pa + poff), db, id_o, (j > 0 || k > 0) ? 1u : 0u);
+          mma(tO, desc_kmajor(pa + (uint32_t)(2 * kBox) + poff), db, id_o, 1u);
+        }
+        commit(o_done);
+        commit(&kv_empty[s]);
+      };
+      for (int j = 0; j < nkt; ++j) {
+        const int s = j & 1;
+        if (!wait_bar(&kv_full[s], (uint32_t)((j >> 1) & 1))) atomicOr(a.err, 2);
+        fence_after();
+        const uint32_t ka = smem_u32(smem + kKVOff + (size_t)s * kStage);
+#pragma unroll
+        for (int k = 0; k < kHD / 16; ++k) {  // 16 dims per MMA
+          const uint32_t off = (uint32_t)((k >> 2) * kBox) + (uint32_t)((k & 3) * 32);
+          mma(tS0 + (uint32_t)(s * kKB), desc_kmajor(qa + off), desc_kmajor(ka + off), id_s, k > 0 ? 1u : 0u);
+        }
+        commit(&s_full[s]);
+        if (j > 0) pv(j - 1);
+      }
+      if (nkt > 0) pv(nkt - 1);
+    }
+  } else if (warp >= 4) {
+    // -------------------------------------------------------------- softmax
+    const int r = (warp - 4) * 32 + lane;  // query row of the block = TMEM lane
+    const uint32_t lane_off = (uint32_t)((warp - 4) * 32) << 16;
+    const int qpos = a.pos0 + q0 + r;      // this row sees keys 0 .. qpos
+    const float sl2 = a.scale * kLog2e;
+    float m_run = -INFINITY, l_run = 0.f;
+    for (int j = 0; j < nkt; ++j) {
+      const int s = j & 1;
+      if (!wait_bar(&s_full[s], (uint32_t)((j >> 1) & 1))) atomicOr(a.err, 2);
+      fence_after();
+      uint32_t sv[kKB];
+#pragma unroll
+      for (int c = 0; c < kKB / 32; ++c) tmem_ld32_nowait(tS0 + lane_off + (uint32_t)(s * kKB + 32 * c), sv + 32 * c);
+      tmem_ld_wait();
+      // scaled scores, masked beyond the row's position; the tile's max
+      float mt = -INFINITY;
+      const int kb = j * kKB;
+#pragma unroll
+      for (int c = 0; c < kKB; ++c) {
+        const float x = kb + c <= qpos ? __uint_as_float(sv[c]) * sl2 : -INFINITY;
+        sv[c] = __float_as_uint(x);
+        mt = fmaxf(mt, x);
+      }
+      // the product of the tile before must be done: the P buffer is reused
+      // and O may be rescaled below
+      if (j > 0 && !wait_bar(o_done, (uint32_t)((j - 1) & 1))) atomicOr(a.err, 2);
+      fence_after();
+      // This row's max moves when the tile's max exceeds it by more than 2^8
+      // (or on the first tile); O and l are then rescaled.  tcgen05.ld / st are
+      // warp-collective, so the warp rescales when any of its rows needs it,
+      // the other rows by 1.
+      float alpha = 1.f;
+      if (mt > m_run + kRescale || m_run == -INFINITY) {
+        const float mnew = fmaxf(mt, m_run);
+        if (m_run != -INFINITY) alpha = exp2f(m_run - mnew);
+        if (mnew != -INFINITY) m_run = mnew;
+      }
+      l_run *= alpha;
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+        for (int c = 0; c < kHD / 32; ++c) {
+          uint32_t ov[32];
+          tmem_ld32_nowait(tO + lane_off + (uint32_t)(32 * c), ov);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+          tmem_st32(tO + lane_off + (uint32_t)(32 * c), ov);
+        }
+        tmem_st_wait();
+      }
+      // P = 2^(s - m) as bf16 high and low parts into the K-major,
+      // 128-byte-swizzled buffers
+      uint8_t* pbuf = smem + kPOff;
+      const float msafe = m_run == -INFINITY ? 0.f : m_run;
+      float lsum = 0.f;
+#pragma unroll
+      for (int ch = 0; ch < kKB / 8; ++ch) {  // 16-byte chunks of 8 keys
+        float pe[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          pe[e] = exp2f(__uint_as_float(sv[8 * ch + e]) - msafe);
+          lsum += pe[e];
+        }
+        float plo[8];
+        const uint4 hi = pack16<bf16>(pe);
+        float phi[8];
+        unpack16<bf16>(hi, phi);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) plo[e] = pe[e] - phi[e];
+        const int box = ch >> 3, c8 = ch & 7;
+        const size_t off = box * kBox + r * 128 + ((c8 ^ (r & 7)) << 4);
+        *reinterpret_cast<uint4*>(pbuf + off) = hi;
+        *reinterpret_cast<uint4*>(pbuf + 2 * kBox + off) = pack16<bf16>(plo);
+      }
+      l_run += lsum;
+      // keys past the ones written so far are stale cache rows (possibly not
+      // finite, and 0 * inf would poison the sum): zero them in V
+      if (j == nkt - 1 && kb + kKB > keys_end) {
+        if (!wait_bar(&kv_full[s], (uint32_t)((j >> 1) & 1))) atomicOr(a.err, 2);
+        uint8_t* vt = smem + kKVOff + (size_t)s * kStage + 2 * kBox;
+        const int row0 = keys_end - kb;  // first stale row of the tile
+        for (int i = r; i < (kKB - row0) * 16; i += 128) {  // 16 chunks of 16 bytes per row
+          const int vr = row0 + i / 16, ch = i % 16;
+          *reinterpret_cast<uint4*>(vt + (ch >> 3) * kBox + vr * 128 + (((ch & 7) ^ (vr & 7)) << 4)) =
+              make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+      fence_proxy_async_smem();  // P (and zeroed V rows) are read by the MMA next
+      fence_before();
+      mbar_arrive(&p_full[s]);
+    }
+    // ---- the last product, then O / l in bf16
+    if (nkt > 0 && !wait_bar(o_done, (uint32_t)((nkt - 1) & 1))) atomicOr(a.err, 2);
+    fence_after();
+    const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+    const int row = q0 + r;
+    bf16* out = reinterpret_cast<bf16*>(a.out) + (size_t)row * a.out_row_stride + (size_t)h * kHD;
+#pragma unroll
+    for (int c = 0; c < kHD / 32; ++c) {
+      uint32_t ov[32];
+      tmem_ld32_nowait(tO + lane_off + (uint32_t)(32 * c), ov);
+      tmem_ld_wait();
+      if (row < a.rows) {
+#pragma unroll
+        for (int e = 0; e < 32; e += 8) {
+          float f[8];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) f[t] = __uint_as_float(ov[e + t]) * inv;
+          *reinterpret_cast<uint4*>(out + 32 * c + e) = pack16<bf16>(f);
+        }
+      }
+    }
+  }
+
+  fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512) : "memory");
+  }
+}
+
+// K/V either head-major (positions of one kv head contiguous, the cache's
+// layout: [nkv][positions][hd]) or token-major (the heads of one position
+// contiguous: [positions][nkv][hd]).
+static bool kv_head_major(const AttnRows& a) { return a.kv_tok_stride == kHD && a.kv_head_stride % kHD == 0; }
+static bool kv_token_major(const AttnRows& a) {
+  return a.kv_head_stride == kHD && a.kv_tok_stride % 8 == 0 && a.kv_tok_stride >= (long long)a.nkv * kHD;
+}
+
+bool attn_tc_supported(const AttnRows& a, int dtype) {
+  return dtype == Q2_BF16 && a.hd == kHD && !a.seq_is_row && a.lens == nullptr && a.row_step == 1 &&
+         a.nkv > 0 && a.nh % a.nkv == 0 && a.rows >= 16 && a.base >= 1 && (a.q_row_stride % 8) == 0 &&
+         (kv_head_major(a) || kv_token_major(a)) && (a.out_row_stride % 8) == 0 &&
+         (reinterpret_cast<uintptr_t>(a.q) & 15) == 0 && (reinterpret_cast<uintptr_t>(a.k) & 15) == 0 &&
+         (reinterpret_cast<uintptr_t>(a.v) & 15) == 0 && (reinterpret_cast<uintptr_t>(a.out) & 15) == 0;
+}
+
+q2_status launch_attn_tc(const AttnRows& a, int* err, cudaStream_t st) {
+  if (a.rows == 0) return Q2_OK;
+  const int pos0 = a.base - 1;
+  const long long keys = (long long)pos0 + a.rows;  // keys visible to the last row
+  CUtensorMap tq, tk, tv;
+  // Q as [rows, nh * hd]
+  Q2_TRY(make_tmap_2d_bf16(&tq, a.q, (uint64_t)a.rows, (uint64_t)a.nh * kHD, (uint64_t)a.q_row_stride * 2, kQB,
+                           64, 128));
+  AttnTc p;
+  if (kv_head_major(a)) {
+    // [nkv * positions, hd]: kv head g starts at row g * positions
+    const long long kv_rows = a.kv_head_stride / kHD;
+    Q2_TRY(make_tmap_2d_bf16(&tk, a.k, (uint64_t)a.nkv * kv_rows, kHD, kHD * 2, kKB, 64, 128));
+    Q2_TRY(make_tmap_2d_bf16(&tv, a.v, (uint64_t)a.nkv * kv_rows, kHD, kHD * 2, kKB, 64, 128));
+    p.kv_x_step = 0;
+    p.kv_y_step = (int)kv_rows;
+  } else {
+    // [positions, nkv * hd]: kv head g starts at column g * hd; no row past
+    // the visible keys exists in the map (it reads as zeros)
+    Q2_TRY(make_tmap_2d_bf16(&tk, a.k, (uint64_t)keys, (uint64_t)a.nkv * kHD, (uint64_t)a.kv_tok_stride * 2, kKB,
+                             64, 128));
+    Q2_TRY(make_tmap_2d_bf16(&tv, a.v, (uint64_t)keys, (uint64_t)a.nkv * kHD, (uint64_t)a.kv_tok_stride * 2, kKB,
+                             64, 128));
+    p.kv_x_step = kHD;
+    p.kv_y_step = 0;
+  }
+  p.rows = a.rows;
+  p.nh = a.nh;
+  p.nkv = a.nkv;
+  p.pos0 = pos0;
+  p.scale = a.scale;
+  p.out = a.out;
+  p.out_row_stride = a.out_row_stride;
+  p.err = err;
+  Q2_CUDA_TRY(cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem));
+  dim3 grid((a.rows + kQB - 1) / kQB, a.nh);
+  Q2_LAUNCH(attn_tc_kernel, grid, dim3(kThreads), kSmem, st, false, tq, tk, tv, p);
+  return Q2_OK;
+}
+
+}  // namespace q2

@@ -68,10 +68,16 @@ struct AttnRows {
 int attn_splits(int rows, int nkv, int max_keys);
 size_t attn_scratch_bytes(int rows, int nh, int hd, int nsplit);
 q2_status launch_attention(const AttnRows& a, int nsplit, void* scratch, int dtype,
-                           cudaStream_t st, bool pdl);
+                           cudaStream_t st, bool pdl, int* err = nullptr);
 // Rows of one sequence (prefill), bf16, head dim 128: flash-attention on the
 // tensor cores (launch_attention takes it by itself when it applies).
 bool attn_prefill_mma_supported(const AttnRows& a, int dtype);
 q2_status launch_attn_prefill_mma(const AttnRows& a, cudaStream_t st, bool pdl);
+// The same on the sm_100a tensor cores (tcgen05, TMEM accumulators): K/V
+// head-major or token-major, head dim 128, bf16.  A bounded wait that runs
+// out sets value 2 in *err.  launch_attention takes it when it applies.
+bool attn_tc_supported(const AttnRows& a, int dtype);
+int prefill_attn_impl();
+q2_status launch_attn_tc(const AttnRows& a, int* err, cudaStream_t st);
 
 }  // namespace q2

@@ -309,7 +309,7 @@ q2_status run_layers(q2_model* M, int T, int decode, int seq, int pos0, cudaStre
         a.fixed_seq = seq;
         nsplit = attn_splits(T, m.n_kv_heads, pos0 + T);
       }
-      TIMED(Q2_K_ATTN, launch_attention(a, nsplit, M->attn_scratch, dt, st, pdl));
+      TIMED(Q2_K_ATTN, launch_attention(a, nsplit, M->attn_scratch, dt, st, pdl, M->d_err));
     }
 
     if (tc) {
