@@ -10,15 +10,21 @@ Qwen2-1.5B shape, random-init bf16 weights, batch 1, a 512-token prompt of
 uniform random ids prefilled first (timed separately), then the timed decode
 steps (context 512 + warmup + steps).  Per step the kernels stream all
 3.09 GB of weights, far more than the 126 MB L2, so no L2 flush is needed.
-Extra keys report batch 64 at 4096 context (`b64`, KV filled with N(0,1)),
-the 512-token prefill (`prefill`), the 32768-token prefill (`prefill_long`),
-the tcgen05 GEMM on the prefill linears at 4096 tokens (the model's prefill
-chunk) and 32768 tokens (`prefill_gemms`, fraction of the measured bf16
-peak), per-kernel times inside
-the decode step (`kernels_ms`), the roofline of the gate/up GEMV (`roofline`,
-with the DRAM traffic recorded under `profiles/` while its sources are
-unchanged), the host-buffer entry point end to end (`e2e`), SM clocks during
-the timed region (`clocks`) and the CPU oracle baseline (`cpu_baseline`).
+At batch 1 the step is one kernel launch (the streaming step), so the
+roofline object (`roofline`) is that kernel's: the step's algorithmic bytes
+over its event-timed launch, with the DRAM traffic recorded under
+`profiles/` while its sources are unchanged.  Extra keys report the phases
+of that launch (`phases_us`: critical-path time per phase, from the
+kernel's own global-timer stamps), the other decode paths' step times
+(`paths_ms`), batch 64 at 4096 context (`b64`, KV filled with N(0,1), with a
+per-kernel-class breakdown), the 512-token prefill (`prefill`), the
+32768-token prefill (`prefill_long`), the tcgen05 GEMM on the prefill linears
+at 4096 tokens (the model's prefill chunk, first) and 32768 tokens
+(`prefill_gemms`, fraction of the measured bf16 peak), the host-buffer entry
+point end to end (`e2e`), SM clocks during the timed region (`clocks`) and
+the CPU oracle baseline (`cpu_baseline`).  Fractions of HBM are given against
+the measured copy bandwidth (`frac`) and against the ~8 TB/s datasheet
+figure (`frac_vs_8tbs`).
 
 Multi-GPU: replicas (`--gpus N` under torchrun): every rank decodes its own
 sequences, no data-path collective; the time is the max over ranks.
@@ -49,6 +55,7 @@ WORKLOAD = "qwen2-1.5b-b1-prompt512-decode128"
 WORKLOAD_B64 = "qwen2-1.5b-b64-ctx4096-decode32"
 WORKLOAD_LONG = "qwen2-1.5b-b1-prompt32768-decode64"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DATASHEET_HBM_GBS = 8000.0  # B200 HBM3e, datasheet
 
 
 def peaks():
@@ -168,6 +175,7 @@ def decode_step_bytes(s, batch: int, ctx: float) -> float:
 # traffic figure stands only while these are unchanged.
 KERNEL_SOURCES = {
     "gate_up": ["decode.cu", "decode.h", "common.cuh", "tma.h", "kernels.h"],
+    "stream_step": ["sdecode.cu", "sdecode.h", "common.cuh", "tma.h", "pdecode.h"],
 }
 
 
@@ -243,9 +251,12 @@ def run_reference(args, dist: Dist):
     tps, desc, n = oracle_decode_sample(max_seconds=min(120.0, 1.5 * args.steps),
                                         max_substeps=args.steps)
     wall = time.perf_counter() - t0
+    # A step of this arm is one sub-step (one layer of the token plus 1/28 of the
+    # lm_head), so ms_per_step x steps is the arm's timed run.
     line = {
         "impl": "reference", "metric": METRIC, "value": tps, "unit": "tok/s", "n_gpus": args.gpus,
-        "steps": n, "warmup": args.warmup, "ms_per_step": 1000.0 / tps, "higher_is_better": True,
+        "steps": n, "substeps_per_token": 28, "warmup": args.warmup,
+        "ms_per_step": 1000.0 / tps / 28, "ms_per_token": 1000.0 / tps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64 (bf16 storage)", "data": "synthetic",
         "config": {"workload": WORKLOAD, "batch": 1, "context": 512, "sampled": True},
         "cpu_baseline": {"value": tps, "unit": "tok/s", "cores": 1, "kind": "oracle", "sample": desc},
@@ -281,7 +292,7 @@ def run_ours(args, dist: Dist):
     b64 = not args.no_b64
     max_batch = 64 if b64 else 1
     past64 = synth.WORKLOADS[WORKLOAD_B64]["past"]
-    max_seq = max(prompt_len + args.warmup + args.steps + 64, (past64 + args.b64_steps + 16) if b64 else 0)
+    max_seq = max(prompt_len + args.warmup + args.steps + 128, (past64 + args.b64_steps + 16) if b64 else 0)
     model = q2.Model(shape, max_seq=max_seq, max_batch=max_batch)
     for key in shape.weight_shapes():  # drawn on the GPU tensor by tensor, copied in, freed
         t = synth.weight(shape, key[0], key[1], seed, device="cuda")
@@ -321,9 +332,27 @@ def run_ours(args, dist: Dist):
     ctx_mean = prompt_len + args.warmup + (args.steps - 1) / 2.0
     step_bytes = decode_step_bytes(shape, 1, ctx_mean)
 
-    # ---- per-kernel device times inside the same decode step (instrumented replay)
+    # ---- inside the same decode step: with one launch per step (the streaming
+    # step), the critical-path time of each phase from the kernel's own
+    # global-timer stamps and the launch by CUDA events; otherwise each kernel
+    # class by events around its launches (serialised, isolated)
     last = bufs[(cur + args.steps) % 2]
     ktimes, kernels_per_step = model.time_kernels(last, steps=min(args.steps, 20))
+
+    # ---- the other decode paths of batch 1 on the same model (context)
+    paths_ms = {}
+    for path in ("kernels", "persistent"):
+        try:
+            model.set_decode_path(path)
+        except q2.Q2Error:
+            continue
+        pb = [last.clone(), torch.empty_like(last)]
+        for i in range(3):
+            model.decode_step(pb[i % 2], out=pb[(i + 1) % 2])
+        n_p = 10
+        paths_ms[path] = dist.max(cuda_time_b64(model, pb, n_p)) / n_p
+    model.set_decode_path("auto")
+    model.set_seq_len(0, prompt_len + args.warmup + args.steps)
 
     # ---- e2e: the public host-buffer entry point, H2D ids + D2H next each step
     ids_h = torch.empty(1, dtype=torch.int64).pin_memory()
@@ -362,9 +391,31 @@ def run_ours(args, dist: Dist):
         ms64 = dist.max(cuda_time_b64(model, b64bufs, n64)) / n64
         ctx64 = past64 + 3 + (n64 - 1) / 2.0
         bytes64 = decode_step_bytes(shape, B, ctx64)
+        # per kernel class inside the batch-64 step (events around each launch:
+        # serialised, isolated times), with the HBM rate of the classes whose
+        # bytes are known from the shapes
+        k64, kps64 = model.time_kernels(b64bufs[n64 % 2], steps=3)
+        H, I, qkvd = shape.hidden, shape.intermediate, shape.q_dim + 2 * shape.kv_dim
+        cls_bytes = {"qkv": 2 * (qkvd * H + B * (H + qkvd)), "o": 2 * (H * shape.q_dim + B * 2 * H),
+                     "gate_up": 2 * (2 * I * H + B * (H + I)), "down": 2 * (H * I + B * (I + 2 * H)),
+                     "lm_head": 2 * shape.vocab * H + 4 * B * shape.vocab,
+                     "attn": B * (past64 + 3 + n64 / 2.0) * 2 * shape.kv_dim * 2}
+        breakdown = {}
+        for k, (mean_ms, per) in k64.items():
+            if not per:
+                continue
+            e = {"mean_ms": round(mean_ms, 5), "per_step": per}
+            if k in cls_bytes and mean_ms > 0:
+                e["gbs"] = round(cls_bytes[k] / (mean_ms / 1e3) / 1e9, 1)
+                e["frac"] = round(e["gbs"] / float(peaks()[0]["hbm_gbs"]), 3)
+            breakdown[k] = e
         b64_line = {"workload": WORKLOAD_B64, "batch": B, "value": B * dist.world / (ms64 / 1e3),
                     "unit": "tok/s", "ms_per_step": ms64, "steps": n64,
-                    "achieved_gbs": bytes64 / (ms64 / 1e3) / 1e9, "bytes_per_step": bytes64}
+                    "achieved_gbs": bytes64 / (ms64 / 1e3) / 1e9, "bytes_per_step": bytes64,
+                    "frac": bytes64 / (ms64 / 1e3) / 1e9 / float(peaks()[0]["hbm_gbs"]),
+                    "kernels_ms": {"timing": "CUDA events around each launch of a replayed step "
+                                             "(serialised, isolated: they do not add up to the step)",
+                                   "by_class": breakdown, "kernels_per_step": kps64}}
     clk = clocks.stop()
 
     pk, pk_kind = peaks()
@@ -377,9 +428,35 @@ def run_ours(args, dist: Dist):
     if not args.no_prefill_gemms:
         gemms = {str(t): prefill_gemm_rates(shape, t, float(pk["bf16_tflops"]))
                  for t in (int(x) for x in args.prefill_gemm_tokens.split(","))}
-    gu_ms, gu_n = ktimes["gate_up"]
-    gu_bytes = 2 * shape.intermediate * shape.hidden * 2 + shape.hidden * 2 + 2 * shape.intermediate * 2
-    achieved = gu_bytes / (gu_ms / 1e3) / 1e9 if gu_ms > 0 else None
+    step_gbs = step_bytes / (ms_step / 1e3) / 1e9
+    if kernels_per_step == 1:
+        # one launch per step: that kernel is the roofline's subject
+        launch_ms = ktimes["step"][0]
+        achieved = step_bytes / (launch_ms / 1e3) / 1e9 if launch_ms > 0 else None
+        roofline = {"kernel": "sdecode_kernel (batch-1 streaming step, one launch per step)",
+                    "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                    "frac": (achieved / hbm) if achieved else None,
+                    "frac_vs_8tbs": (achieved / DATASHEET_HBM_GBS) if achieved else None,
+                    "traffic": recorded_traffic("stream_step", WORKLOAD),
+                    "bytes_per_launch": step_bytes, "mean_launch_ms": launch_ms, "peak_kind": pk_kind}
+        kernel_times = {"phases_us": {k: round(v[0] * 1e3, 3) for k, v in ktimes.items()
+                                      if v[1] and k != "step"},
+                        "phases_timing": "critical path per phase instance inside the one launch "
+                                         "(latest end of the phase minus latest end of the phase "
+                                         "before, global-timer stamps)"}
+    else:
+        gu_ms, gu_n = ktimes["gate_up"]
+        gu_bytes = 2 * shape.intermediate * shape.hidden * 2 + shape.hidden * 2 + 2 * shape.intermediate * 2
+        achieved = gu_bytes / (gu_ms / 1e3) / 1e9 if gu_ms > 0 else None
+        roofline = {"kernel": "gate_up", "bound": "hbm", "achieved": achieved, "peak": hbm,
+                    "unit": "GB/s", "frac": (achieved / hbm) if achieved else None,
+                    "frac_vs_8tbs": (achieved / DATASHEET_HBM_GBS) if achieved else None,
+                    "traffic": recorded_traffic("gate_up", WORKLOAD),
+                    "bytes_per_launch": gu_bytes, "mean_launch_ms": gu_ms, "peak_kind": pk_kind}
+        kernel_times = {"kernels_ms": {k: {"mean_ms": round(v[0], 5), "per_step": v[1]}
+                                       for k, v in ktimes.items() if v[1]},
+                        "kernels_timing": "CUDA events around each launch of a replayed step "
+                                          "(serialised, isolated: they do not add up to the step)"}
     line = {
         "metric": METRIC,
         "value": 1 * dist.world / (ms_step / 1e3),
@@ -397,14 +474,12 @@ def run_ours(args, dist: Dist):
                    "context": f"{prompt_len + args.warmup}..{prompt_len + args.warmup + args.steps}",
                    "l2": "no flush: each step streams 3.09 GB of weights (> 126 MB L2)",
                    "parallelism": f"replicas x{dist.world}"},
-        "step_roofline": {"bytes_per_step": step_bytes, "achieved_gbs": step_bytes / (ms_step / 1e3) / 1e9,
-                          "peak_gbs": hbm, "frac": step_bytes / (ms_step / 1e3) / 1e9 / hbm,
+        "step_roofline": {"bytes_per_step": step_bytes, "achieved_gbs": step_gbs,
+                          "peak_gbs": hbm, "frac": step_gbs / hbm, "frac_vs_8tbs": step_gbs / DATASHEET_HBM_GBS,
                           "peak_kind": pk_kind},
-        "roofline": {"kernel": "gate_up", "bound": "hbm", "achieved": achieved, "peak": hbm,
-                     "unit": "GB/s", "frac": (achieved / hbm) if achieved else None,
-                     "traffic": recorded_traffic("gate_up", WORKLOAD),
-                     "bytes_per_launch": gu_bytes, "mean_launch_ms": gu_ms, "peak_kind": pk_kind},
-        "kernels_ms": {k: {"mean_ms": round(v[0], 5), "per_step": v[1]} for k, v in ktimes.items() if v[1]},
+        "roofline": roofline,
+        **kernel_times,
+        "paths_ms": paths_ms,
         "gpu_launches": kernels_per_step * args.steps,
         "kernels_per_step": kernels_per_step,
         "prefill": {"tokens": prompt_len, "ms": pre_ms, "tok_s": prompt_len / (pre_ms / 1e3)},

@@ -610,6 +610,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     phase_w(p, layers, ph, bid, G, pw);
     unsigned long long* ctr = p.ctrace ? p.ctrace + ((size_t)ph * G + bid) * 4 : nullptr;
     if (ctr && ct == 0) ctr[0] = gtimer();
+    if (p.trace && ct == 0) {  // the phase's start (latest, and CTA 0's)
+      const unsigned long long t = gtimer();
+      atomicMax(&p.trace[ph * 4 + 3], t);
+      if (bid == 0) p.trace[ph * 4 + 1] = t;
+    }
     uint4 nwr[NCH];    // the RMSNorm weight pieces of this phase (loaded before its input)
     float xr[NCH][8];  // short-row phases: this lane's pieces lane + 32 i of the input vector
 

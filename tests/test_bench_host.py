@@ -42,10 +42,14 @@ def test_recorded_traffic_is_tied_to_the_kernel_sources():
     sources hash to the value stored with it."""
     import json
     b = _bench()
-    rec = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))[f"gate_up@{b.WORKLOAD}"]
-    t = b.recorded_traffic("gate_up", b.WORKLOAD)
-    if rec["src_hash"] == b.kernel_src_hash("gate_up"):
-        assert t == rec["dram_bytes_per_launch"]
-    else:
-        assert t is None
-    assert b.recorded_traffic("gate_up", "another-workload") is None
+    recs = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
+    assert recs
+    for key, rec in recs.items():
+        kernel, workload = key.split("@")
+        assert kernel in b.KERNEL_SOURCES, key
+        t = b.recorded_traffic(kernel, workload)
+        if rec["src_hash"] == b.kernel_src_hash(kernel):
+            assert t == rec["dram_bytes_per_launch"]
+        else:
+            assert t is None
+        assert b.recorded_traffic(kernel, "another-workload") is None
