@@ -396,12 +396,20 @@ static bool kv_token_major(const AttnRows& a) {
   return a.kv_head_stride == kHD && a.kv_tok_stride % 8 == 0 && a.kv_tok_stride >= (long long)a.nkv * kHD;
 }
 
+// K and V of the rows' sequence (a.fixed_seq)
+static const bf16* seq_k(const AttnRows& a) {
+  return reinterpret_cast<const bf16*>(a.k) + (size_t)a.fixed_seq * a.kv_seq_stride;
+}
+static const bf16* seq_v(const AttnRows& a) {
+  return reinterpret_cast<const bf16*>(a.v) + (size_t)a.fixed_seq * a.kv_seq_stride;
+}
+
 bool attn_tc_supported(const AttnRows& a, int dtype) {
   return dtype == Q2_BF16 && a.hd == kHD && !a.seq_is_row && a.lens == nullptr && a.row_step == 1 &&
-         a.nkv > 0 && a.nh % a.nkv == 0 && a.rows >= 16 && a.base >= 1 && (a.q_row_stride % 8) == 0 &&
-         (kv_head_major(a) || kv_token_major(a)) && (a.out_row_stride % 8) == 0 &&
-         (reinterpret_cast<uintptr_t>(a.q) & 15) == 0 && (reinterpret_cast<uintptr_t>(a.k) & 15) == 0 &&
-         (reinterpret_cast<uintptr_t>(a.v) & 15) == 0 && (reinterpret_cast<uintptr_t>(a.out) & 15) == 0;
+         a.nkv > 0 && a.nh % a.nkv == 0 && a.rows >= 16 && a.base >= 1 && a.fixed_seq >= 0 &&
+         (a.q_row_stride % 8) == 0 && (kv_head_major(a) || kv_token_major(a)) && (a.out_row_stride % 8) == 0 &&
+         (reinterpret_cast<uintptr_t>(a.q) & 15) == 0 && (reinterpret_cast<uintptr_t>(seq_k(a)) & 15) == 0 &&
+         (reinterpret_cast<uintptr_t>(seq_v(a)) & 15) == 0 && (reinterpret_cast<uintptr_t>(a.out) & 15) == 0;
 }
 
 q2_status launch_attn_tc(const AttnRows& a, int* err, cudaStream_t st) {
@@ -416,17 +424,17 @@ q2_status launch_attn_tc(const AttnRows& a, int* err, cudaStream_t st) {
   if (kv_head_major(a)) {
     // [nkv * positions, hd]: kv head g starts at row g * positions
     const long long kv_rows = a.kv_head_stride / kHD;
-    Q2_TRY(make_tmap_2d_bf16(&tk, a.k, (uint64_t)a.nkv * kv_rows, kHD, kHD * 2, kKB, 64, 128));
-    Q2_TRY(make_tmap_2d_bf16(&tv, a.v, (uint64_t)a.nkv * kv_rows, kHD, kHD * 2, kKB, 64, 128));
+    Q2_TRY(make_tmap_2d_bf16(&tk, seq_k(a), (uint64_t)a.nkv * kv_rows, kHD, kHD * 2, kKB, 64, 128));
+    Q2_TRY(make_tmap_2d_bf16(&tv, seq_v(a), (uint64_t)a.nkv * kv_rows, kHD, kHD * 2, kKB, 64, 128));
     p.kv_x_step = 0;
     p.kv_y_step = (int)kv_rows;
   } else {
     // [positions, nkv * hd]: kv head g starts at column g * hd; no row past
     // the visible keys exists in the map (it reads as zeros)
-    Q2_TRY(make_tmap_2d_bf16(&tk, a.k, (uint64_t)keys, (uint64_t)a.nkv * kHD, (uint64_t)a.kv_tok_stride * 2, kKB,
-                             64, 128));
-    Q2_TRY(make_tmap_2d_bf16(&tv, a.v, (uint64_t)keys, (uint64_t)a.nkv * kHD, (uint64_t)a.kv_tok_stride * 2, kKB,
-                             64, 128));
+    Q2_TRY(make_tmap_2d_bf16(&tk, seq_k(a), (uint64_t)keys, (uint64_t)a.nkv * kHD, (uint64_t)a.kv_tok_stride * 2,
+                             kKB, 64, 128));
+    Q2_TRY(make_tmap_2d_bf16(&tv, seq_v(a), (uint64_t)keys, (uint64_t)a.nkv * kHD, (uint64_t)a.kv_tok_stride * 2,
+                             kKB, 64, 128));
     p.kv_x_step = kHD;
     p.kv_y_step = 0;
   }

@@ -218,6 +218,25 @@ def mid():
     return shape, synth.model_weights(shape, 77, device="cuda")
 
 
+def test_batched_prefill_matches_each_sequence_alone(mid):
+    """Prefill of several sequences in one call: each sequence's attention
+    reads its own K/V cache (sequence 1 has enough rows for the tensor-core
+    attention, sequence 2 too few), so its logits match a prefill of that
+    sequence alone."""
+    shape, w = mid
+    gm = q2.Model(shape, max_seq=128, max_batch=4)
+    gm.load(w)
+    lens = [20, 33, 7]
+    prompts = [synth.prompt_ids(shape, n, 40 + b, seq=b) for b, n in enumerate(lens)]
+    _, lg = gm.prefill(torch.cat(prompts).cuda(), lens, want_logits=True)
+    lg = lg.cpu()
+    for b, pr in enumerate(prompts):
+        gm.reset_kv()
+        _, one = gm.prefill(pr.cuda(), [lens[b]], want_logits=True)
+        assert_bf16_logits(one[0].cpu(), lg[b], f"sequence {b} alone vs batched")
+    gm.check_error()
+
+
 def test_prefill_plus_decode_equals_longer_prefill(mid):
     shape, w = mid
     gm = q2.Model(shape, max_seq=128)
