@@ -243,6 +243,19 @@ __device__ __forceinline__ void mma16816(float* c, uint32_t a0, uint32_t a2, uin
 
 __device__ __forceinline__ int phase_kind(int L, int ph) { return ph == 5 * L ? PH_HEAD : ph % 5; }
 
+// Two warp sums with one reduction tree: lane 0 returns the sum of u over the
+// warp, lane 16 the sum of v.  Each total is added up in the same order as
+// warp_sum's butterfly (lane l with l ^ 16, then ^ 8, ^ 4, ^ 2, ^ 1), so the
+// results are bitwise those of two warp_sum calls.
+__device__ __forceinline__ float warp_sum_pair(float u, float v, int lane) {
+  const bool hi = (lane & 16) != 0;
+  float keep = hi ? v : u;
+  keep += __shfl_xor_sync(0xffffffffu, hi ? u : v, 16);
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) keep += __shfl_xor_sync(0xffffffffu, keep, o);
+  return keep;
+}
+
 // The weight rows a CTA streams in one phase: rows [r0, r1) of w [N][K], in
 // stages of rs whole rows.  Rows are dealt out in contiguous blocks of whole
 // units: a RoPE pair for q/k/v (one tagged word of q, k or v), two rows for o
@@ -461,96 +474,154 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int c = ct; c < n / 8; c += kCT) reinterpret_cast<uint4*>(xbuf)[c] = __ldcg(reinterpret_cast<const uint4*>(src) + c);
     csync();
   };
-  // xr = this lane's pieces of xbuf, bf16(rmsnorm(xbuf) * nw) if nw is given:
-  // every warp normalises the whole vector itself.
-  auto input_regs = [&](bool norm, const uint4 (&nwr)[NCH], float (&xr)[NCH][8]) {
+  // xr = this lane's pieces of xbuf, bf16(rmsnorm(xbuf) * nw) if nw is given,
+  // as packed bf16 (every value is a bf16 either way): every warp normalises
+  // the whole vector itself.
+  auto input_regs = [&](bool norm, const uint4 (&nwr)[NCH], uint4 (&xr)[NCH]) {
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) xr[i] = reinterpret_cast<const uint4*>(xbuf)[lane + 32 * i];
+    if (!norm) return;
     float ss = 0.f;
 #pragma unroll
     for (int i = 0; i < NCH; ++i) {
-      unpack16<bf16>(reinterpret_cast<const uint4*>(xbuf)[lane + 32 * i], xr[i]);
+      float f[8];
+      unpack16<bf16>(xr[i], f);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) ss = fmaf(xr[i][e], xr[i][e], ss);
+      for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
     }
-    if (!norm) return;
     ss = warp_sum(ss);
     const float inv = rsqrtf(ss / (float)(NCH * 256) + p.eps);
 #pragma unroll
     for (int i = 0; i < NCH; ++i) {
-      float wf[8];
+      float f[8], wf[8];
+      unpack16<bf16>(xr[i], f);
       unpack16<bf16>(nwr[i], wf);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) xr[i][e] = round_st<bf16>(xr[i][e] * inv * wf[e]);
+      for (int e = 0; e < 8; ++e) f[e] = round_st<bf16>(f[e] * inv * wf[e]);
+      xr[i] = pack16<bf16>(f);
     }
   };
 
-  // The stages of one short-row phase: warp w takes rows w, w + 8, ... of each
-  // stage; the row result goes to yrow (or, for the lm_head, to the logits).
-  auto consume_short = [&](const PW& pw, bool head, const float (&xr)[NCH][8]) {
-    for (int r = pw.r0; r < pw.r1; r += pw.rs, ++gs) {
-      const int slot = c_slot;
-      const uint32_t par = c_par;
-      if (++c_slot == RING) {
-        c_slot = 0;
-        c_par ^= 1u;
-      }
+  // The next stage of the ring: waits until it has landed, returns its slot.
+  auto take_stage = [&]() {
+    const int slot = c_slot;
+    const uint32_t par = c_par;
+    if (++c_slot == RING) {
+      c_slot = 0;
+      c_par ^= 1u;
+    }
+    ++gs;
+    if (!bwait(&full[slot], par, dl, p.sync) && lane == 0) atomicOr(p.err, 2);
+    return slot;
+  };
+
+  // The lm_head's stages, one at a time: warp w takes rows w, w + 8, ... of
+  // each stage; the logits are written and the warp's argmax kept.
+  auto consume_head = [&](const PW& pw, const uint4 (&xr)[NCH]) {
+    for (int r = pw.r0; r < pw.r1; r += pw.rs) {
+      const int s0 = take_stage();
       const int n = min(pw.rs, pw.r1 - r);
-      if (!bwait(&full[slot], par, dl, p.sync) && lane == 0) atomicOr(p.err, 2);
-      const uint8_t* st = ring + (size_t)slot * kSB;
+      const uint8_t* st = ring + (size_t)s0 * kSB;
       for (int rr = warp; rr < n; rr += kCW) {
         const uint4* wrow = reinterpret_cast<const uint4*>(st + (size_t)rr * pw.K * 2);
         float a[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int i = 0; i < NCH; ++i) {
-          float wf[8];
-          unpack16<bf16>(wrow[lane + 32 * i], wf);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) a[e & 3] = fmaf(wf[e], xr[i][e], a[e & 3]);
-        }
-        const float y = warp_sum((a[0] + a[1]) + (a[2] + a[3]));
-        if (head) {
-          const int row = r + rr;
-          if (lane == 0) p.logits[row] = y;
-          if (am_better(y, row, best_v, best_i)) {
-            best_v = y;
-            best_i = row;
-          }
-        } else if (lane == 0) {
-          yrow[r + rr - pw.r0] = y;
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[slot]);
-    }
-  };
-
-  // The stages of the down phase: one row per stage, warp w takes column
-  // pieces [w * cpw, (w + 1) * cpw) of it.
-  auto consume_long = [&](const PW& pw, const uint4 (&xs)[NQ]) {
-    const int cpw = pw.K / 8 / kCW;
-    for (int r = pw.r0; r < pw.r1; r += pw.rs, ++gs) {
-      const int slot = c_slot;
-      const uint32_t par = c_par;
-      if (++c_slot == RING) {
-        c_slot = 0;
-        c_par ^= 1u;
-      }
-      if (!bwait(&full[slot], par, dl, p.sync) && lane == 0) atomicOr(p.err, 2);
-      const uint4* wrow = reinterpret_cast<const uint4*>(ring + (size_t)slot * kSB) + warp * cpw;
-      float a[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int q = 0; q < NQ; ++q) {
-        if (lane + 32 * q < cpw) {
           float wf[8], xf[8];
-          unpack16<bf16>(wrow[lane + 32 * q], wf);
-          unpack16<bf16>(xs[q], xf);
+          unpack16<bf16>(wrow[lane + 32 * i], wf);
+          unpack16<bf16>(xr[i], xf);
 #pragma unroll
           for (int e = 0; e < 8; ++e) a[e & 3] = fmaf(wf[e], xf[e], a[e & 3]);
         }
+        const float y = warp_sum((a[0] + a[1]) + (a[2] + a[3]));
+        const int row = r + rr;
+        if (lane == 0) p.logits[row] = y;
+        if (am_better(y, row, best_v, best_i)) {
+          best_v = y;
+          best_i = row;
+        }
       }
-      const float y = warp_sum((a[0] + a[1]) + (a[2] + a[3]));
-      if (lane == 0) part[warp * kDMax + (r - pw.r0)] = y;
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[slot]);
+      if (lane == 0) mbar_arrive(&empty[s0]);
+    }
+  };
+
+  // The stages of the other short-row phases, two at a time: warp w takes
+  // rows w, w + 8, ... of each stage, row rr of both stages together, so that
+  // the two rows' loads and products overlap and share one reduction tree;
+  // the row results go to yrow.
+  auto consume_short = [&](const PW& pw, const uint4 (&xr)[NCH]) {
+    for (int r = pw.r0; r < pw.r1; r += 2 * pw.rs) {
+      const bool two = r + pw.rs < pw.r1;
+      const int s0 = take_stage();
+      const int s1 = two ? take_stage() : s0;
+      const int n0 = min(pw.rs, pw.r1 - r);
+      const int n1 = two ? min(pw.rs, pw.r1 - r - pw.rs) : 0;
+      const uint8_t* st0 = ring + (size_t)s0 * kSB;
+      const uint8_t* st1 = ring + (size_t)s1 * kSB;
+      for (int rr = warp; rr < n0; rr += kCW) {
+        const bool has1 = rr < n1;  // warp-uniform
+        const uint4* w0 = reinterpret_cast<const uint4*>(st0 + (size_t)rr * pw.K * 2);
+        const uint4* w1 = reinterpret_cast<const uint4*>(st1 + (size_t)(has1 ? rr : 0) * pw.K * 2);
+        float a[4] = {0.f, 0.f, 0.f, 0.f}, b[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int i = 0; i < NCH; ++i) {
+          float wf[8], vf[8], xf[8];
+          unpack16<bf16>(w0[lane + 32 * i], wf);
+          unpack16<bf16>(has1 ? w1[lane + 32 * i] : make_uint4(0u, 0u, 0u, 0u), vf);
+          unpack16<bf16>(xr[i], xf);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            a[e & 3] = fmaf(wf[e], xf[e], a[e & 3]);
+            b[e & 3] = fmaf(vf[e], xf[e], b[e & 3]);
+          }
+        }
+        // lane 0: row rr of the first stage, lane 16: of the second
+        const float y = warp_sum_pair((a[0] + a[1]) + (a[2] + a[3]), (b[0] + b[1]) + (b[2] + b[3]), lane);
+        if (lane == 0) yrow[r + rr - pw.r0] = y;
+        if (lane == 16 && has1) yrow[r + pw.rs + rr - pw.r0] = y;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&empty[s0]);
+        if (two) mbar_arrive(&empty[s1]);
+      }
+    }
+  };
+
+  // The stages of the down phase, two at a time: one row per stage, warp w
+  // takes column pieces [w * cpw, (w + 1) * cpw) of both rows.
+  auto consume_long = [&](const PW& pw, const float (&xf)[NQ][8]) {
+    const int cpw = pw.K / 8 / kCW;
+    for (int r = pw.r0; r < pw.r1; r += 2 * pw.rs) {
+      const bool two = r + pw.rs < pw.r1;  // warp-uniform
+      const int s0 = take_stage();
+      const int s1 = two ? take_stage() : s0;
+      const uint4* w0 = reinterpret_cast<const uint4*>(ring + (size_t)s0 * kSB) + warp * cpw;
+      const uint4* w1 = reinterpret_cast<const uint4*>(ring + (size_t)s1 * kSB) + warp * cpw;
+      float a[4] = {0.f, 0.f, 0.f, 0.f}, b[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) {
+        if (lane + 32 * q < cpw) {
+          float wf[8], vf[8];
+          unpack16<bf16>(w0[lane + 32 * q], wf);
+          unpack16<bf16>(two ? w1[lane + 32 * q] : make_uint4(0u, 0u, 0u, 0u), vf);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            a[e & 3] = fmaf(wf[e], xf[q][e], a[e & 3]);
+            b[e & 3] = fmaf(vf[e], xf[q][e], b[e & 3]);
+          }
+        }
+      }
+      // lane 0: the first stage's row, lane 16: the second's
+      const float y = warp_sum_pair((a[0] + a[1]) + (a[2] + a[3]), (b[0] + b[1]) + (b[2] + b[3]), lane);
+      if (lane == 0) part[warp * kDMax + (r - pw.r0)] = y;
+      if (lane == 16 && two) part[warp * kDMax + (r + pw.rs - pw.r0)] = y;
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&empty[s0]);
+        if (two) mbar_arrive(&empty[s1]);
+      }
     }
   };
 
@@ -616,7 +687,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (bid == 0) p.trace[ph * 4 + 1] = t;
     }
     uint4 nwr[NCH];    // the RMSNorm weight pieces of this phase (loaded before its input)
-    float xr[NCH][8];  // short-row phases: this lane's pieces lane + 32 i of the input vector
+    uint4 xr[NCH];     // short-row phases: this lane's pieces lane + 32 i of the input vector
 
     // ---- what does not depend on the previous phase, before waiting for it
     if (kind == PH_QKV) {
@@ -902,7 +973,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       prefetch_tiles(l + 1);
     } else if (kind == PH_DOWN) {
-      uint4 xs[NQ];  // this lane's pieces of the warp's column slice of s (bf16)
+      uint4 xs[NQ];  // this lane's pieces of the warp's column slice of s (bf16), then as fp32
+      float xf[NQ][8];
       const int cpw = pw.K / 8 / kCW;
       {
         const uint64_t* sbase = p.ll.s + (size_t)(warp * cpw + lane) * 4;
@@ -924,7 +996,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (ctr && ct == 0) ctr[1] = gtimer();
-      consume_long(pw, xs);
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) unpack16<bf16>(xs[q], xf[q]);
+      consume_long(pw, xf);
     } else {  // the short-row phases: q/k/v, o, gate/up, lm_head
       if (kind == PH_QKV && l == 0) {
         // layer 0: the embedding row (an id outside the vocabulary sets bit 0 of
@@ -946,7 +1020,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (ctr && ct == 0) ctr[1] = gtimer();
       input_regs(kind != PH_O, nwr, xr);
-      consume_short(pw, kind == PH_HEAD, xr);
+      if (kind == PH_HEAD)
+        consume_head(pw, xr);
+      else
+        consume_short(pw, xr);
     }
 
     // ---- phase epilogue from the parked row results and staged operands
