@@ -33,6 +33,7 @@ constexpr int kAT = 64;                // attention keys per tile
 constexpr int kHD = 128;               // head dim of this kernel
 constexpr int kTile = kAT * kHD * 2;   // one K (or V) tile
 constexpr int kAGMax = 8;              // query heads per kv head
+constexpr int kPS = 72;                // keys per row of the attention P buffers (64 + padding)
 constexpr int kYMax = 256;             // rows per CTA of a short-row phase (parked row results)
 constexpr int kDMax = 64;              // rows per CTA of the o and down phases
 constexpr int kQMax = 64;              // q/k/v rows per CTA (staged epilogue operands)
@@ -56,7 +57,7 @@ constexpr size_t kPart = kYrow + (size_t)kYMax * 4;            // [kCW][kDMax] d
 constexpr size_t kXres = kPart + (size_t)kCW * kDMax * 4;       // [kDMax] this CTA's residual rows
 constexpr size_t kEbias = kXres + (size_t)kDMax * 4;           // [kQMax] q/k/v bias of this CTA's rows
 constexpr size_t kEcs = kEbias + (size_t)kQMax * 4;            // [kQMax / 2] RoPE (cos, sin) per row pair
-constexpr size_t kMlw = kEcs + (size_t)kQMax / 2 * 8;          // [kCW][kAGMax][2] per-warp attention max, sum
+constexpr size_t kMlw = kEcs + (size_t)kQMax / 2 * 8;          // [128] attention: per-head rescale, merge weights
 constexpr size_t kAmv = kMlw + (size_t)kCW * kAGMax * 2 * 4;   // [kCW] per-warp argmax values
 constexpr size_t kAmi = kAmv + (size_t)kCW * 8;                // [kCW] per-warp argmax indices (8-aligned)
 constexpr size_t kXbuf = kAmi + (size_t)kCW * 8;               // [kHMax] bf16: the phase's input vector
@@ -66,6 +67,14 @@ constexpr size_t kAbar = kKvn + 2 * (size_t)kHD * 2;           // abar[2]
 constexpr size_t kFlags = kAbar + 2 * 8;                       // [8] ints
 constexpr size_t kRing = (kFlags + 8 * 4 + 1023) / 1024 * 1024;  // [ring][kSB] weight ring
 static_assert(kAmi % 8 == 0 && kXbuf % 16 == 0 && kAbar % 8 == 0, "shared-memory alignment");
+// the attention phase borrows: xbuf for the partial scores, yrow + part for P
+// (high and low), mlw for the rescale and merge weights, the tiles for the
+// merger's staged partials
+static_assert(2 * kAT * kAGMax * 4 <= kHMax * 2, "attention scores");
+static_assert(kPart == kYrow + (size_t)kYMax * 4 && 2 * kAGMax * kPS * 2 <= kYMax * 4 + kCW * kDMax * 4, "P");
+static_assert(kAGMax + kSplitMax + 1 <= kCW * kAGMax * 2, "merge weights");
+static_assert((size_t)kSplitMax * (kHD + 2) * 4 <= 4 * (size_t)kTile, "merger staging");
+static_assert(kAT == 64 && kHD == 16 * kCW && kAGMax <= kCW, "attention work split");
 }  // namespace sl
 
 struct SLay {
@@ -200,6 +209,36 @@ __device__ __forceinline__ void get_lines(const Poll& pl, const uint64_t* base, 
   }
 }
 
+// The same with each line's address given.
+template <int N>
+__device__ __forceinline__ void get_lines_at(const Poll& pl, const uint64_t* const (&at)[N], uint32_t mask,
+                                             uint32_t tag, uint2 (&out)[N]) {
+  uint32_t pending = mask;
+  uint64_t t0 = 0;
+  for (unsigned it = 0; pending; ++it) {
+    uint4 v[N];
+#pragma unroll
+    for (int i = 0; i < N; ++i)
+      if ((pending >> i) & 1u)
+        asm volatile("ld.volatile.global.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(v[i].x), "=r"(v[i].y), "=r"(v[i].z), "=r"(v[i].w)
+                     : "l"(at[i])
+                     : "memory");
+#pragma unroll
+    for (int i = 0; i < N; ++i)
+      if ((pending >> i) & 1u) {
+        out[i] = make_uint2(v[i].x, v[i].z);
+        if (v[i].y == tag && v[i].w == tag) pending &= ~(1u << i);
+      }
+    if (!pending) break;
+    if (it == 0) t0 = gtimer();
+    if ((it & 7u) == 7u && pl.stop(t0)) {
+      pl.fail();
+      break;
+    }
+  }
+}
+
 __device__ __forceinline__ uint32_t bf2_bits(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&v);
@@ -231,14 +270,14 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t&
                : "r"(addr));
 }
 
-// c += A . B for one m16n8k16 tile (bf16 in, fp32 accumulate); A rows 8..15 are
-// zero, so only a0 (row g, k pair 2t) and a2 (row g, k pair 2t + 8) are given.
-__device__ __forceinline__ void mma16816(float* c, uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
+// c += A . B for one m16n8k16 tile with all four A registers given.
+__device__ __forceinline__ void mma16816_a4(float* c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                            uint32_t b0, uint32_t b1) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
       "{%8, %9}, {%0, %1, %2, %3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 __device__ __forceinline__ int phase_kind(int L, int ph) { return ph == 5 * L ? PH_HEAD : ph % 5; }
@@ -625,8 +664,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   };
 
-  // ---- attention work items: (kv head, split) pairs; a split spans at least
-  // two tiles and its range follows from the length.
+  // ---- attention work items: (kv head, split) pairs, item = split * nkv + kv
+  // head.  A split is a run of tiles of 64 keys: one tile per split while the
+  // splits fit (at most nsplit per kv head, and the last nh CTAs are left to
+  // the mergers), so a short context is spread one tile per CTA.
   struct AItem {
     int gq, split, ntiles, tps, t0, t1, nact;
   };
@@ -635,7 +676,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     a.gq = item % p.nkv;
     a.split = item / p.nkv;
     a.ntiles = (alen + kAT - 1) / kAT;
-    const int active = min(p.nsplit, (a.ntiles + 1) / 2);
+    const int smax = max(1, min(p.nsplit, (G - p.nh) / p.nkv));
+    const int active = min(smax, a.ntiles);
     a.tps = (a.ntiles + active - 1) / active;
     a.t0 = a.split * a.tps;
     a.t1 = min(a.t0 + a.tps, a.ntiles);
@@ -707,26 +749,35 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---- the phase's input, then its weight stages
     if (kind == PH_ATTN) {
-      // Tensor-core attention over each tile: warp (grp, wq) takes keys
-      // [16 wq, 16 wq + 16) and output dims [64 grp, 64 grp + 64): scores
-      // q_h . k_j by mma.sync (the kv head's query heads on M, keys on N, head
-      // dims on K; both groups compute them), online softmax in fp32, P . V by
-      // mma.sync (P in a bf16 high and low part) for the group's dims.  The
-      // four warps of a group are merged in shared memory; the first split of
-      // a kv head then merges the other splits' partials and publishes.
-      const int grp = warp >> 2, wq = warp & 3;
-      const int fr = lane >> 2, fc = lane & 3;  // mma fragment coordinates
+      // Attention over the cache on the tensor cores with the keys on M.  Per
+      // tile of 64 keys: S^T = K q^T (warp w: keys 16 (w % 4) .. + 15 against
+      // the kv head's query heads on N, over head dims 64 (w / 4) .. + 63; the
+      // two halves are added in shared memory), an online softmax per query
+      // head (warp h takes head h: keys lane and lane + 32), then O^T += V^T P
+      // (warp w: head dims 16 w .. + 15; P as bf16 high and low parts, so the
+      // probabilities keep ~16 significant bits).  The split's partial
+      // (unnormalised o, max, sum per query head) goes out from the
+      // accumulators; CTA G - 1 - h merges the splits of query head h.
+      const int g8 = lane >> 2, t4 = lane & 3;  // mma fragment coordinates
       const int mi = lane >> 3, mr = lane & 7;  // ldmatrix: lane addresses row mr of matrix mi
       const float sl2 = p.scale * kLog2e;
       const uint32_t tq = rtag(ph - 1), ta = wtag(ph);
+      float* Sp = reinterpret_cast<float*>(xbuf);  // [2 dim halves][64 keys][8 heads], heads swizzled
+      bf16* Ph = reinterpret_cast<bf16*>(yrow);     // [8 heads][kPS keys] P, high part
+      bf16* Pl = Ph + kAGMax * kPS;                  // low part
+      float* alph = mlw;                             // [8] this tile's rescale per head
+      float* ew = mlw + kAGMax;                      // [kSplitMax + 1] merger: split weights, 1 / sum
+      auto sp_at = [](int dh, int key, int h) { return (dh * kAT + key) * kAGMax + (h ^ ((key >> 2) & 7)); };
+      const size_t hstride = kHD + 2;  // words per (split, head) partial
       for (int item = bid; item < aitems; item += G) {
         const AItem a = attn_item(item);
         if (a.t0 >= a.t1) continue;
         const int nt = a.t1 - a.t0;
+        const bool last = a.t1 == a.ntiles;  // this split holds the new position
         const int pre = item == bid ? s_flags[2] : 0;
         if (ct == 0)
           for (int q = pre; q < 2 && q < nt; ++q) tile_issue(l, a.gq, a.t0 + q, ac + q);
-        // q of the kv head's query heads and the new K/V row, from the tagged words
+        // q of the kv head's query heads (and the new K/V row), from the tagged words
         for (int v = ct; v < Gq * half / 2; v += kCT) {
           const int hh = v / (half / 2), j = 2 * (v % (half / 2));
           const uint2 d = pl.get2(p.ll.q + (size_t)(a.gq * Gq + hh) * half + j, tq);
@@ -736,241 +787,206 @@ __global__ void __launch_bounds__(kThreads, 1)
           qh[j + 1] = __ushort_as_bfloat16((unsigned short)(d.y & 0xffffu));
           qh[j + 1 + half] = __ushort_as_bfloat16((unsigned short)(d.y >> 16));
         }
-        for (int v = ct; v < half; v += kCT) {  // K pairs, then V pairs
-          const int sel = v / (half / 2), j = 2 * (v % (half / 2));
-          const uint2 d = pl.get2(p.ll.kv + (size_t)(sel * p.nkv + a.gq) * half + j, tq);
-          bf16* r = kvn + sel * kHD;
-          r[j] = __ushort_as_bfloat16((unsigned short)(d.x & 0xffffu));
-          r[j + half] = __ushort_as_bfloat16((unsigned short)(d.x >> 16));
-          r[j + 1] = __ushort_as_bfloat16((unsigned short)(d.y & 0xffffu));
-          r[j + 1 + half] = __ushort_as_bfloat16((unsigned short)(d.y >> 16));
-        }
+        if (last)
+          for (int v = ct; v < half; v += kCT) {  // K pairs, then V pairs
+            const int sel = v / (half / 2), j = 2 * (v % (half / 2));
+            const uint2 d = pl.get2(p.ll.kv + (size_t)(sel * p.nkv + a.gq) * half + j, tq);
+            bf16* r = kvn + sel * kHD;
+            r[j] = __ushort_as_bfloat16((unsigned short)(d.x & 0xffffu));
+            r[j + half] = __ushort_as_bfloat16((unsigned short)(d.x >> 16));
+            r[j + 1] = __ushort_as_bfloat16((unsigned short)(d.y & 0xffffu));
+            r[j + 1 + half] = __ushort_as_bfloat16((unsigned short)(d.y >> 16));
+          }
         csync();
         if (ctr && ct == 0 && item == bid) ctr[1] = gtimer();  // attention: q and the new K/V row in
-        // A fragments of the query heads (bf16, unscaled); rows fr >= Gq are zero
-        uint32_t qa[8][2];
+        const int kq = 16 * (warp & 3), dh = warp >> 2;
+        // B fragments of q^T (head dims x query heads) for this warp's dim half;
+        // heads past the group are zero
+        uint32_t qb[4][2];
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const bf16* qrow = qst + (fr < Gq ? fr : 0) * kHD + 16 * kk + 2 * fc;
-          qa[kk][0] = fr < Gq ? *reinterpret_cast<const uint32_t*>(qrow) : 0u;
-          qa[kk][1] = fr < Gq ? *reinterpret_cast<const uint32_t*>(qrow + 8) : 0u;
+        for (int ks = 0; ks < 4; ++ks) {
+          const bf16* qrow = qst + (g8 < Gq ? g8 : 0) * kHD + 64 * dh + 16 * ks + 2 * t4;
+          qb[ks][0] = g8 < Gq ? *reinterpret_cast<const uint32_t*>(qrow) : 0u;
+          qb[ks][1] = g8 < Gq ? *reinterpret_cast<const uint32_t*>(qrow + 8) : 0u;
         }
-        float o[8][4];
-#pragma unroll
-        for (int n = 0; n < 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-        float m_run = -INFINITY, l_run = 0.f;
+        // O^T accumulators: head dims 16 warp + g8 (+ 8) x heads 2 t4 (+ 1), from
+        // the high and the low part of P
+        float oh[4] = {0.f, 0.f, 0.f, 0.f}, ol[4] = {0.f, 0.f, 0.f, 0.f};
+        float m_run = -INFINITY, l_run = 0.f;  // softmax of head `warp`
         for (int i = 0; i < nt; ++i) {
           const int li = ac + i, stg = li & 1;
           const int t = a.t0 + i;
           if (!bwait(&abar[stg], (uint32_t)((li >> 1) & 1), dl) && lane == 0) atomicOr(p.err, 2);
           uint8_t* tk = tiles + (size_t)stg * 2 * kTile;
+          uint8_t* tv = tk + kTile;
           if (t == a.ntiles - 1) {
             // the tile holding the new position: its row comes from the
-            // published K/V (the cache row may have been read before it existed)
+            // published K/V (the cache row may have been read before it
+            // existed), and the rows after it are stale cache rows (possibly not
+            // finite: their scores are masked, their V rows zeroed)
+            const int r = pos - t * kAT;
             if (warp == 0) {
-              const int r = pos - t * kAT, c = lane & 15;
-              uint8_t* dst = tk + (lane < 16 ? 0 : kTile) + (c >> 3) * 8192 + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+              const int c = lane & 15;
+              uint8_t* dst = (lane < 16 ? tk : tv) + (c >> 3) * 8192 + r * 128 + (((c & 7) ^ (r & 7)) << 4);
               *reinterpret_cast<uint4*>(dst) = reinterpret_cast<const uint4*>(kvn + (lane < 16 ? 0 : kHD))[c];
-              fence_proxy_async_smem();
+            }
+            for (int c = ct; c < (kAT - 1 - r) * 16; c += kCT) {
+              const int vr = r + 1 + c / 16, ch = c % 16;
+              *reinterpret_cast<uint4*>(tv + (ch >> 3) * 8192 + vr * 128 + (((ch & 7) ^ (vr & 7)) << 4)) =
+                  make_uint4(0u, 0u, 0u, 0u);
             }
             csync();
           }
-          const uint32_t kt = smem_u32(tk);
-          const uint32_t vt = kt + (uint32_t)kTile;
-          // ---- scores of this warp's 16 keys: s0 keys +0..7, s1 keys +8..15, each
-          // summed over the head dims in two independent chains (even and odd
-          // k-steps) to halve the dependent MMA latency
-          float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+          const uint32_t ka = smem_u32(tk), va = smem_u32(tv);
+          // ---- S^T, keys kq .. kq + 15 x heads, over this warp's dim half
           {
-            float s0b[4] = {0.f, 0.f, 0.f, 0.f}, s1b[4] = {0.f, 0.f, 0.f, 0.f};
-            const int key = wq * 16 + ((mi >> 1) << 3) + mr;
+            float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const int dim = 16 * kk + ((mi & 1) << 3);
+            for (int ks = 0; ks < 4; ++ks) {
               uint32_t r0, r1, r2, r3;
-              ldsm_x4(kt + (uint32_t)((dim >> 6) * 8192) + swz_off(key, dim & 63), r0, r1, r2, r3);
-              mma16816((kk & 1) ? s0b : s0, qa[kk][0], qa[kk][1], r0, r1);
-              mma16816((kk & 1) ? s1b : s1, qa[kk][0], qa[kk][1], r2, r3);
+              ldsm_x4(ka + (uint32_t)(dh * 8192) + swz_off(kq + mr + ((mi & 1) << 3), 16 * ks + ((mi >> 1) << 3)),
+                      r0, r1, r2, r3);
+              mma16816_a4((ks & 1) ? sb : sa, r0, r1, r2, r3, qb[ks][0], qb[ks][1]);
             }
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              s0[e] += s0b[e];
-              s1[e] += s1b[e];
-            }
+            Sp[sp_at(dh, kq + g8, 2 * t4)] = sa[0] + sb[0];
+            Sp[sp_at(dh, kq + g8, 2 * t4 + 1)] = sa[1] + sb[1];
+            Sp[sp_at(dh, kq + g8 + 8, 2 * t4)] = sa[2] + sb[2];
+            Sp[sp_at(dh, kq + g8 + 8, 2 * t4 + 1)] = sa[3] + sb[3];
           }
-          // ---- online softmax for head fr over keys kb + 2fc, +1 and kb + 8 + 2fc, +1
-          const int kb = t * kAT + wq * 16 + 2 * fc;
-          float sc[4] = {s0[0] * sl2, s0[1] * sl2, s1[0] * sl2, s1[1] * sl2};
-          if (kb >= alen) sc[0] = -INFINITY;
-          if (kb + 1 >= alen) sc[1] = -INFINITY;
-          if (kb + 8 >= alen) sc[2] = -INFINITY;
-          if (kb + 9 >= alen) sc[3] = -INFINITY;
-          float mloc = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
-          mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
-          mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 2));
-          const float mnew = fmaxf(m_run, mloc);
-          const float msafe = mnew == -INFINITY ? 0.f : mnew;
-          const float alpha = exp2f(m_run - msafe);
-          float pr[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) pr[e] = exp2f(sc[e] - msafe);
-          float psum = (pr[0] + pr[1]) + (pr[2] + pr[3]);
-          psum += __shfl_xor_sync(0xffffffffu, psum, 1);
-          psum += __shfl_xor_sync(0xffffffffu, psum, 2);
-          l_run = l_run * alpha + psum;
-          m_run = mnew;
-#pragma unroll
-          for (int n = 0; n < 8; ++n) {
-            o[n][0] *= alpha;
-            o[n][1] *= alpha;
-          }
-          // P in two bf16 parts, hi = bf16(p) and lo = bf16(p - hi), so that the
-          // probabilities keep ~16 significant bits through the bf16 MMA.
-          float ph_[4], pl_[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            ph_[e] = __bfloat162float(__float2bfloat16_rn(pr[e]));
-            pl_[e] = pr[e] - ph_[e];
-          }
-          const uint32_t pa0 = bf2_bits(ph_[0], ph_[1]), pa2 = bf2_bits(ph_[2], ph_[3]);
-          const uint32_t pb0 = bf2_bits(pl_[0], pl_[1]), pb2 = bf2_bits(pl_[2], pl_[3]);
-          // positions past the sequence hold stale cache rows (possibly not
-          // finite): their V entries are zeroed, as 0 * inf would poison the sum
-          const uint32_t vm0 = (kb < alen ? 0x0000ffffu : 0u) | (kb + 1 < alen ? 0xffff0000u : 0u);
-          const uint32_t vm1 = (kb + 8 < alen ? 0x0000ffffu : 0u) | (kb + 9 < alen ? 0xffff0000u : 0u);
-          // ---- O += P . V over the same 16 keys, the group's 64 dims, 16 (two
-          // n8 tiles) per ldmatrix
+          csync();
+          // ---- online softmax of head `warp` over the tile's keys lane, lane + 32
           {
-            const int key = wq * 16 + ((mi & 1) << 3) + mr;
-#pragma unroll
-            for (int nd = 0; nd < 4; ++nd) {
-              const int dim = 64 * grp + 16 * nd + ((mi >> 1) << 3);
-              uint32_t r0, r1, r2, r3;
-              ldsm_x4_t(vt + (uint32_t)((dim >> 6) * 8192) + swz_off(key, dim & 63), r0, r1, r2, r3);
-              r0 &= vm0;
-              r1 &= vm1;
-              r2 &= vm0;
-              r3 &= vm1;
-              mma16816(o[2 * nd], pa0, pa2, r0, r1);
-              mma16816(o[2 * nd], pb0, pb2, r0, r1);
-              mma16816(o[2 * nd + 1], pa0, pa2, r2, r3);
-              mma16816(o[2 * nd + 1], pb0, pb2, r2, r3);
+            const int h = warp;
+            bf16* ph = Ph + h * kPS;
+            bf16* plo = Pl + h * kPS;
+            if (h < Gq) {
+              const int kb = t * kAT;
+              float s0 = (Sp[sp_at(0, lane, h)] + Sp[sp_at(1, lane, h)]) * sl2;
+              float s1 = (Sp[sp_at(0, lane + 32, h)] + Sp[sp_at(1, lane + 32, h)]) * sl2;
+              if (kb + lane >= alen) s0 = -INFINITY;
+              if (kb + lane + 32 >= alen) s1 = -INFINITY;
+              // key kb is always visible, so the tile's max is finite
+              const float mnew = fmaxf(m_run, warp_max(fmaxf(s0, s1)));
+              const float alpha = exp2f(m_run - mnew);  // 0 on the first tile
+              const float p0 = exp2f(s0 - mnew), p1 = exp2f(s1 - mnew);
+              l_run = l_run * alpha + warp_sum(p0 + p1);
+              m_run = mnew;
+              const bf16 h0 = __float2bfloat16_rn(p0), h1 = __float2bfloat16_rn(p1);
+              ph[lane] = h0;
+              ph[lane + 32] = h1;
+              plo[lane] = __float2bfloat16_rn(p0 - __bfloat162float(h0));
+              plo[lane + 32] = __float2bfloat16_rn(p1 - __bfloat162float(h1));
+              if (lane == 0) alph[h] = alpha;
+            } else {  // no such head: zero P
+              const bf16 z = __float2bfloat16_rn(0.f);
+              ph[lane] = ph[lane + 32] = plo[lane] = plo[lane + 32] = z;
+              if (lane == 0) alph[h] = 1.f;
             }
           }
-          csync();  // every warp is done with this stage
-          if (ct == 0 && i + 2 < nt) tile_issue(l, a.gq, t + 2, li + 2);
+          csync();
+          // ---- O^T += V^T P for head dims 16 warp .. + 15
+          {
+            const float a0 = alph[2 * t4], a1 = alph[2 * t4 + 1];
+            oh[0] *= a0;
+            oh[1] *= a1;
+            oh[2] *= a0;
+            oh[3] *= a1;
+            ol[0] *= a0;
+            ol[1] *= a1;
+            ol[2] *= a0;
+            ol[3] *= a1;
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+              uint32_t r0, r1, r2, r3;
+              ldsm_x4_t(va + (uint32_t)((warp >> 2) * 8192) +
+                            swz_off(16 * ks + mr + ((mi >> 1) << 3), 16 * (warp & 3) + ((mi & 1) << 3)),
+                        r0, r1, r2, r3);
+              const int kk = g8 * kPS + 16 * ks + 2 * t4;
+              mma16816_a4(oh, r0, r1, r2, r3, *reinterpret_cast<const uint32_t*>(Ph + kk),
+                          *reinterpret_cast<const uint32_t*>(Ph + kk + 8));
+              mma16816_a4(ol, r0, r1, r2, r3, *reinterpret_cast<const uint32_t*>(Pl + kk),
+                          *reinterpret_cast<const uint32_t*>(Pl + kk + 8));
+            }
+          }
+          if (i + 2 < nt) {
+            csync();  // every warp is done with this stage
+            if (ct == 0) tile_issue(l, a.gq, t + 2, li + 2);
+          }
         }
         ac += nt;
         if (ctr && ct == 0 && item == bid) ctr[2] = gtimer();  // attention: tiles done
-
-        // ---- the four warps of each group (max, sum, unnormalised output),
-        // merged; the tile buffers are free now (every tile of the item was
-        // waited on)
-        float* Ow = reinterpret_cast<float*>(tiles);  // [kCW][kAGMax][64]
-        if (fr < Gq) {
+        // ---- this split's partial, from the accumulators
+        uint64_t* pb = p.ll.part + (size_t)(a.gq * kSplitMax + a.split) * Gq * hstride;
+        const int d0 = 16 * warp + g8;
 #pragma unroll
-          for (int n = 0; n < 8; ++n) {
-            float* dst = Ow + ((size_t)warp * kAGMax + fr) * 64 + 8 * n + 2 * fc;
-            dst[0] = o[n][0];
-            dst[1] = o[n][1];
-          }
-          if (fc == 0) {
-            mlw[(warp * kAGMax + fr) * 2] = m_run;
-            mlw[(warp * kAGMax + fr) * 2 + 1] = l_run;
+        for (int e = 0; e < 2; ++e) {
+          const int hh = 2 * t4 + e;
+          if (hh < Gq) {
+            ll_put(pb + hh * hstride + d0, __float_as_uint(oh[e] + ol[e]), ta);
+            ll_put(pb + hh * hstride + d0 + 8, __float_as_uint(oh[2 + e] + ol[2 + e]), ta);
           }
         }
-        csync();
-        // thread ct takes dims (2 dp, 2 dp + 1) of head hh for items i = ct, ct + kCT
-        // (Gq * half <= 2 kCT): this split's (max, sum, output) of them
-        float cM[2], cL[2], cO0[2], cO1[2];
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          const int i = ct + kCT * k;
-          cM[k] = -INFINITY;
-          cL[k] = cO0[k] = cO1[k] = 0.f;
-          if (i >= Gq * half) continue;
-          const int hh = i / half, d = 2 * (i % half), w0 = 4 * (d >> 6);
-          float M = -INFINITY;
-#pragma unroll
-          for (int w = w0; w < w0 + 4; ++w) M = fmaxf(M, mlw[(w * kAGMax + hh) * 2]);
-          const float Ms = M == -INFINITY ? 0.f : M;
-#pragma unroll
-          for (int w = w0; w < w0 + 4; ++w) {
-            const float e = exp2f(mlw[(w * kAGMax + hh) * 2] - Ms);
-            const float* ow = Ow + ((size_t)w * kAGMax + hh) * 64 + (d & 63);
-            cO0[k] = fmaf(e, ow[0], cO0[k]);
-            cO1[k] = fmaf(e, ow[1], cO1[k]);
-            cL[k] = fmaf(e, mlw[(w * kAGMax + hh) * 2 + 1], cL[k]);
-          }
-          cM[k] = M;
-        }
-        const size_t hstride = kHD + 2;  // words per (split, head)
-        if (a.split > 0) {  // a partial for the first split of this kv head
-          uint64_t* pb = p.ll.part + (size_t)(a.gq * kSplitMax + a.split) * Gq * hstride;
-#pragma unroll
-          for (int k = 0; k < 2; ++k) {
-            const int i = ct + kCT * k;
-            if (i >= Gq * half) continue;
-            const int hh = i / half, d = 2 * (i % half);
-            ll_put2(pb + hh * hstride + d, __float_as_uint(cO0[k]), __float_as_uint(cO1[k]), ta);
-            if (d == 0) ll_put2(pb + hh * hstride + kHD, __float_as_uint(cM[k]), __float_as_uint(cL[k]), ta);
-          }
-        } else {
-          // The first split merges the others in split order:
-          // o = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s.  Their partials
-          // are staged into the (free) tile buffer a chunk of splits at a
-          // time, each thread polling its share of the chunk's lines at once.
-          const int chunk = (int)(4 * (size_t)kTile / (Gq * hstride * 4));  // splits that fit the buffer
-          float* pst = reinterpret_cast<float*>(tiles);
-          const uint64_t* pb0 = p.ll.part + (size_t)(a.gq * kSplitMax) * Gq * hstride;
-          for (int s0 = 1; s0 < a.nact; s0 += chunk) {
-            const int ns = min(chunk, a.nact - s0);
-            const int nlines = ns * Gq * (int)hstride / 2;
-            csync();  // the buffer's previous contents (partials, earlier chunk) are read
-            for (int l0 = 0; l0 < nlines; l0 += 4 * kCT) {
-              uint2 got[4];
-              uint32_t mask = 0;
-#pragma unroll
-              for (int k = 0; k < 4; ++k)
-                if (l0 + ct + kCT * k < nlines) mask |= 1u << k;
-              get_lines<4>(pl, pb0 + (size_t)s0 * Gq * hstride + 2 * (size_t)l0, 2 * 2 * kCT, 2 * (size_t)ct,
-                           2 * (size_t)(ct + kCT), mask, rtag(ph), got);
-#pragma unroll
-              for (int k = 0; k < 4; ++k)
-                if ((mask >> k) & 1u)
-                  reinterpret_cast<uint2*>(pst)[l0 + ct + kCT * k] =
-                      make_uint2(got[k].x, got[k].y);
-            }
-            csync();
-#pragma unroll
-            for (int k = 0; k < 2; ++k) {
-              const int i = ct + kCT * k;
-              if (i >= Gq * half) continue;
-              const int hh = i / half, d = 2 * (i % half);
-              for (int sp = 0; sp < ns; ++sp) {
-                const float* ps = pst + ((size_t)sp * Gq + hh) * hstride;
-                const float ms = ps[kHD], lsp = ps[kHD + 1];
-                const float Mn = fmaxf(cM[k], ms);
-                const float ea = exp2f(cM[k] - Mn), eb = exp2f(ms - Mn);
-                cO0[k] = cO0[k] * ea + ps[d] * eb;
-                cO1[k] = cO1[k] * ea + ps[d + 1] * eb;
-                cL[k] = cL[k] * ea + lsp * eb;
-                cM[k] = Mn;
-              }
-            }
-          }
-#pragma unroll
-          for (int k = 0; k < 2; ++k) {
-            const int i = ct + kCT * k;
-            if (i >= Gq * half) continue;
-            const int hh = i / half, dp = i % half;
-            const float inv = cL[k] > 0.f ? 1.f / cL[k] : 0.f;
-            ll_put(p.ll.att + (size_t)(a.gq * Gq + hh) * half + dp, bf2_bits(cO0[k] * inv, cO1[k] * inv), ta);
-          }
-        }
-        fence_proxy_async_smem();  // the tile buffer is a TMA destination again later
-        csync();
+        if (warp < Gq && lane == 0)
+          ll_put2(pb + warp * hstride + kHD, __float_as_uint(m_run), __float_as_uint(l_run), ta);
+        csync();  // the next item's q, scores and P overwrite this one's
       }
+      // ---- the merge of query head mh = G - 1 - bid over its splits:
+      // o = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s, M = max_s m_s.  The
+      // partials are staged in the tile buffers (free: every tile this CTA
+      // issued has been waited on and read).
+      const int mh = G - 1 - bid;
+      if (mh >= 0 && mh < p.nh) {
+        const AItem a = attn_item(0);
+        const int gq = mh / Gq, hh = mh % Gq;
+        const int lps = (int)(hstride / 2);  // 16-byte lines per split partial
+        const int nlines = a.nact * lps;
+        float* pst = reinterpret_cast<float*>(tiles);  // [nact][hstride]
+        const uint64_t* pb0 = p.ll.part + (size_t)gq * kSplitMax * Gq * hstride + (size_t)hh * hstride;
+        for (int l0 = 0; l0 < nlines; l0 += 4 * kCT) {
+          const uint64_t* at[4];
+          uint32_t mask = 0;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int L = l0 + ct + kCT * k;
+            at[k] = pb0;
+            if (L < nlines) {
+              mask |= 1u << k;
+              at[k] = pb0 + (size_t)(L / lps) * Gq * hstride + 2 * (L % lps);
+            }
+          }
+          uint2 got[4];
+          get_lines_at<4>(pl, at, mask, rtag(ph), got);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            if ((mask >> k) & 1u) reinterpret_cast<uint2*>(pst)[l0 + ct + kCT * k] = got[k];
+        }
+        csync();
+        if (warp == 0) {
+          float M = -INFINITY;
+          for (int sp = lane; sp < a.nact; sp += 32) M = fmaxf(M, pst[sp * hstride + kHD]);
+          M = warp_max(M);
+          float Ls = 0.f;
+          for (int sp = lane; sp < a.nact; sp += 32) {
+            const float e = exp2f(pst[sp * hstride + kHD] - M);
+            ew[sp] = e;
+            Ls = fmaf(e, pst[sp * hstride + kHD + 1], Ls);
+          }
+          Ls = warp_sum(Ls);
+          if (lane == 0) ew[kSplitMax] = Ls > 0.f ? 1.f / Ls : 0.f;
+        }
+        csync();
+        if (ct < half) {
+          float o0 = 0.f, o1 = 0.f;
+          for (int sp = 0; sp < a.nact; ++sp) {
+            o0 = fmaf(ew[sp], pst[sp * hstride + 2 * ct], o0);
+            o1 = fmaf(ew[sp], pst[sp * hstride + 2 * ct + 1], o1);
+          }
+          const float inv = ew[kSplitMax];
+          ll_put(p.ll.att + (size_t)mh * half + ct, bf2_bits(o0 * inv, o1 * inv), ta);
+        }
+      }
+      fence_proxy_async_smem();  // the tile buffers are TMA destinations again
+      csync();
       prefetch_tiles(l + 1);
     } else if (kind == PH_DOWN) {
       uint4 xs[NQ];  // this lane's pieces of the warp's column slice of s (bf16), then as fp32
@@ -1241,6 +1257,10 @@ q2_status launch_sdecode(const SDecode& p, const CUtensorMap& kmap, const CUtens
   const long long o_rows = (long long)(p.H / 2 + G - 1) / G * 2;
   if (qkv_rows > kQMax || gu_rows > kYMax || o_rows > kYMax || o_rows > kDMax) {
     set_error("streaming decode: too many rows per CTA for this device");
+    return Q2_ERR_SHAPE;
+  }
+  if (G < p.nh + p.nkv) {  // a merger CTA per query head, and an attention CTA per kv head besides
+    set_error("streaming decode: fewer SMs than query plus kv heads");
     return Q2_ERR_SHAPE;
   }
   auto kern = sdecode_kernel<kNCH, kNQ>;

@@ -32,9 +32,11 @@
 // Phases (l = layer):
 //   QKV(l)  RMSNorm (layer 0: embedding row) -> q/k/v rows, bias, RoPE; q and
 //           the new K/V row published, K/V appended to the cache
-//   ATTN(l) split attention over the cache (K/V tiles by TMA, the tile holding
-//           the new position patched with the published row); the first split
-//           of a kv head merges the others' partials and publishes the output
+//   ATTN(l) split attention over the cache, one tile of 64 keys per CTA while
+//           the splits fit (K/V tiles by TMA a layer ahead, the tile holding the
+//           new position patched with the published row); each split publishes
+//           its partial, and CTA G - 1 - h merges query head h's partials and
+//           publishes its output
 //   O(l)    o rows, residual add (x published)
 //   GU(l)   RMSNorm -> gate/up row pairs, SwiGLU (s published)
 //   DOWN(l) down rows (each split over the warps by columns), residual add
