@@ -555,6 +555,81 @@ def cuda_time_b64(model, bufs, n):
     return s.elapsed_time(e)
 
 
+PROFILE_CASES = ("stream-small", "stream-full", "gemm4096", "attn-chunk", "b64-layer")
+
+
+def run_profile_case(case: str):
+    """A small, self-contained run of one kernel's workload for ncu captures
+    (the summaries under profiles/ name these commands).  Prints one line of
+    what ran; no timing is reported."""
+    import dataclasses
+    import qwen2_decode_step_b200 as q2
+    torch.cuda.init()
+    shape = synth.QWEN2_1P5B
+    if case in ("stream-small", "stream-full"):
+        # batch-1 streaming steps after a 512-token prompt: 4 layers and a
+        # 32000-row vocabulary (0.47 GB of weights, above L2), or the full model
+        if case == "stream-small":
+            shape = dataclasses.replace(shape, n_layers=4, vocab=32000)
+        seed = synth.WORKLOADS[WORKLOAD]["seed"]
+        m = q2.Model(shape, max_seq=640, max_batch=1)
+        for key in shape.weight_shapes():
+            t = synth.weight(shape, key[0], key[1], seed, device="cuda")
+            m.load_weight(key[0], key[1], t)
+            del t
+        m.set_decode_path("stream")
+        m.set_graphs(False)
+        nxt = m.prefill(synth.prompt_ids(shape, 512, seed, device="cuda"), [512])
+        for _ in range(6):
+            nxt = m.decode_step(nxt)
+        torch.cuda.synchronize()
+        m.check_error()
+        m.close()
+        print(f"{case}: {shape.n_layers} layers, 6 streaming steps at context 512..517")
+    elif case == "gemm4096":
+        out = prefill_gemm_rates(shape, 4096, 1.0, reps=1)
+        print("gemm4096: the q/k/v, o, gate/up and down linears at M = 4096 (3 warm-up + 1 call each):",
+              {k: (v["N"], v["K"]) for k, v in out.items()})
+    elif case == "attn-chunk":
+        # the last 4096-row chunk of the 32768-token prompt: rows at positions
+        # 28672.. over 32768 keys, K/V token-major (the operator's layout)
+        import math
+        S, T, nh, nkv, hd = 4096, 32768, shape.n_heads, shape.n_kv_heads, shape.head_dim
+        q = synth.normal((S, nh, hd), 1.0, 11, "bf16").cuda()
+        k = synth.normal((T, nkv, hd), 1.0, 12, "bf16").cuda()
+        v = synth.normal((T, nkv, hd), 1.0, 13, "bf16").cuda()
+        o = torch.empty((S, nh, hd), dtype=torch.bfloat16, device="cuda")
+        for _ in range(3):
+            q2.q2_self_attention(o, q, k, v, 1.0 / math.sqrt(hd))
+        torch.cuda.synchronize()
+        q2.q2_check_device_error()
+        print(f"attn-chunk: {S} query rows x {T} keys, {nh} heads / {nkv} kv heads, 3 calls")
+    elif case == "b64-layer":
+        # one full-size decoder layer at batch 64 over 4096 cached positions
+        one = dataclasses.replace(shape, n_layers=1)
+        wl = synth.WORKLOADS[WORKLOAD_B64]
+        B, past = wl["batch"], wl["past"]
+        m = q2.Model(one, max_seq=past + 16, max_batch=B)
+        for key in one.weight_shapes():
+            t = synth.weight(one, key[0], key[1], wl["seed"], device="cuda")
+            m.load_weight(key[0], key[1], t)
+            del t
+        for b in range(B):
+            kk, vv = synth.kv_fill(one, past, wl["seed"], 0, b, device="cuda")
+            gk, gv = m.kv_cache(0, b)
+            gk[:, :past].copy_(kk.permute(1, 0, 2))
+            gv[:, :past].copy_(vv.permute(1, 0, 2))
+            m.set_seq_len(b, past)
+        m.set_graphs(False)
+        ids = synth.uniform_ids(B, one.vocab, wl["seed"] + 7, device="cuda")
+        for _ in range(4):
+            ids = m.decode_step(ids)
+        torch.cuda.synchronize()
+        m.check_error()
+        m.close()
+        print(f"b64-layer: one decoder layer + head, batch {B}, context {past}..{past + 3}, 4 steps")
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -571,7 +646,12 @@ def main():
                     help="token counts at which the prefill linears are timed: the model's prefill "
                          "chunk (4096) and the whole 32768-token prompt as one product")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--profile", choices=PROFILE_CASES,
+                    help="run one small kernel workload for an ncu capture and exit (no bench line)")
     args = ap.parse_args()
+    if args.profile:
+        run_profile_case(args.profile)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     dist = Dist()

@@ -68,6 +68,7 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = gtimer();
   for (;;) {
+#pragma unroll 1
     for (int i = 0; i < 64; ++i)
       if (mbar_try_wait(bar, parity)) return true;
     if (gtimer() - t0 > kDeadlineNs) return false;
@@ -276,18 +277,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int s = j & 1;
       if (!wait_bar(&s_full[s], (uint32_t)((j >> 1) & 1))) atomicOr(a.err, 2);
       fence_after();
-      uint32_t sv[kKB];
-#pragma unroll
-      for (int c = 0; c < kKB / 32; ++c) tmem_ld32_nowait(tS0 + lane_off + (uint32_t)(s * kKB + 32 * c), sv + 32 * c);
-      tmem_ld_wait();
-      // scaled scores, masked beyond the row's position; the tile's max
+      // the tile's max of the scaled scores, masked beyond the row's position,
+      // 32 columns at a time (the row is read again below: short loops keep
+      // the softmax warps' code small enough to stay in the instruction cache)
       float mt = -INFINITY;
       const int kb = j * kKB;
+#pragma unroll 1
+      for (int c = 0; c < kKB / 32; ++c) {
+        uint32_t sv[32];
+        tmem_ld32_nowait(tS0 + lane_off + (uint32_t)(s * kKB + 32 * c), sv);
+        tmem_ld_wait();
 #pragma unroll
-      for (int c = 0; c < kKB; ++c) {
-        const float x = kb + c <= qpos ? __uint_as_float(sv[c]) * sl2 : -INFINITY;
-        sv[c] = __float_as_uint(x);
-        mt = fmaxf(mt, x);
+        for (int e = 0; e < 32; ++e)
+          mt = fmaxf(mt, kb + 32 * c + e <= qpos ? __uint_as_float(sv[e]) * sl2 : -INFINITY);
       }
       // the product of the tile before must be done: the P buffer is reused
       // and O may be rescaled below
@@ -305,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       l_run *= alpha;
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll
+#pragma unroll 1
         for (int c = 0; c < kHD / 32; ++c) {
           uint32_t ov[32];
           tmem_ld32_nowait(tO + lane_off + (uint32_t)(32 * c), ov);
@@ -321,24 +323,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint8_t* pbuf = smem + kPOff;
       const float msafe = m_run == -INFINITY ? 0.f : m_run;
       float lsum = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < kKB / 32; ++c) {
+        uint32_t sv[32];
+        tmem_ld32_nowait(tS0 + lane_off + (uint32_t)(s * kKB + 32 * c), sv);
+        tmem_ld_wait();
 #pragma unroll
-      for (int ch = 0; ch < kKB / 8; ++ch) {  // 16-byte chunks of 8 keys
-        float pe[8];
+        for (int q = 0; q < 4; ++q) {  // 16-byte chunks of 8 keys
+          float pe[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          pe[e] = exp2f(__uint_as_float(sv[8 * ch + e]) - msafe);
-          lsum += pe[e];
+          for (int e = 0; e < 8; ++e) {
+            const int col = 32 * c + 8 * q + e;
+            const float x = kb + col <= qpos ? __uint_as_float(sv[8 * q + e]) * sl2 : -INFINITY;
+            pe[e] = exp2f(x - msafe);
+            lsum += pe[e];
+          }
+          float plo[8];
+          const uint4 hi = pack16<bf16>(pe);
+          float phi[8];
+          unpack16<bf16>(hi, phi);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) plo[e] = pe[e] - phi[e];
+          const int ch = 4 * c + q, box = ch >> 3, c8 = ch & 7;
+          const size_t off = box * kBox + r * 128 + ((c8 ^ (r & 7)) << 4);
+          *reinterpret_cast<uint4*>(pbuf + off) = hi;
+          *reinterpret_cast<uint4*>(pbuf + 2 * kBox + off) = pack16<bf16>(plo);
         }
-        float plo[8];
-        const uint4 hi = pack16<bf16>(pe);
-        float phi[8];
-        unpack16<bf16>(hi, phi);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) plo[e] = pe[e] - phi[e];
-        const int box = ch >> 3, c8 = ch & 7;
-        const size_t off = box * kBox + r * 128 + ((c8 ^ (r & 7)) << 4);
-        *reinterpret_cast<uint4*>(pbuf + off) = hi;
-        *reinterpret_cast<uint4*>(pbuf + 2 * kBox + off) = pack16<bf16>(plo);
       }
       l_run += lsum;
       // keys past the ones written so far are stale cache rows (possibly not
@@ -363,7 +373,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
     const int row = q0 + r;
     bf16* out = reinterpret_cast<bf16*>(a.out) + (size_t)row * a.out_row_stride + (size_t)h * kHD;
-#pragma unroll
+#pragma unroll 1
     for (int c = 0; c < kHD / 32; ++c) {
       uint32_t ov[32];
       tmem_ld32_nowait(tO + lane_off + (uint32_t)(32 * c), ov);

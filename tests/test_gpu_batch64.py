@@ -7,7 +7,11 @@ per sequence and kv head).
 The oracle decodes sampled sequences one by one over the same cache:
 * layer by layer with teacher forcing (each layer's sampled rows fed the
   oracle's input for that layer; rows are independent sequences), within the
-  per-layer bound;
+  per-layer bound, then the head (final RMSNorm, lm_head, argmax) on the
+  oracle's final state: logits within the bf16 bound, the token bit-exact
+  against the oracle's argmax of the same fp32 logits (and equal to the
+  oracle's own token when its top two logits are further apart than the
+  logit bound);
 * the whole step free-running for sampled sequences, within the long-context
   free-running bound (twice the oracle's own fp32-accumulation drift at
   32768 positions, an upper bound for 4096).
@@ -19,7 +23,8 @@ import pytest
 import oracle
 import qwen2_decode_step_b200 as q2
 import synth
-from tol import assert_bf16_logits_long_context, assert_layer_close
+import torch
+from tol import assert_bf16_logits, assert_bf16_logits_long_context, assert_layer_close
 
 pytestmark = pytest.mark.gpu
 
@@ -85,6 +90,19 @@ def test_batch64_decode_layerwise_teacher_forced(b64):
             x_ref[b] = y_ref
         del om
         x = y
+    # the head on the oracle's final state of each sampled sequence
+    for b in SAMPLED:
+        h = oracle.rms_norm(x_ref[b], wc[("final_norm", -1)], shape.eps)
+        lg_ref = oracle.linear(h, wc[("lm_head", -1)], None, out_dtype=torch.float32)[0]
+        nxt_ref = int(oracle.argmax(lg_ref)[0][0])
+        nxt, lg = g1.head(x_ref[b].cuda())
+        lg = lg[0].cpu()
+        assert_bf16_logits(lg, lg_ref, f"head, sequence {b}")
+        assert int(nxt[0]) == int(oracle.argmax(lg)[0][0]), f"sequence {b}: argmax of the GPU's logits"
+        top2 = torch.topk(lg_ref, 2).values
+        if float(top2[0] - top2[1]) > 5e-2:
+            assert int(nxt[0]) == nxt_ref, f"sequence {b}: token"
+    g1.check_error()
 
 
 def test_batch64_decode_step_free_running(b64):
