@@ -3,7 +3,7 @@
 // output accumulators in tensor memory, operands in 128-byte-swizzled shared
 // memory, K/V tiles by TMA.
 //
-// One CTA per (128 query rows, query head); 256 threads:
+// One CTA per (128 query rows, query head); 384 threads:
 //   warp 0     TMA: the Q block once (two 64-dim boxes), then K and V tiles
 //              of 128 keys into a two-stage ring
 //   warp 1     allocates tensor memory; one thread issues the MMAs:
@@ -18,13 +18,15 @@
 //              in the order S_0, S_1, O += P_0 V_0, S_2, O += P_1 V_1, ...,
 //              so a tile's scores are computed while the softmax of the tile
 //              before runs
-//   warps 4-7  softmax: thread r owns query row r (TMEM lane r).  It reads its
-//              row of S_j, applies the scale and the causal mask, keeps the
-//              running max m and sum l (O is rescaled only when the max grows
-//              by more than 2^8, so most tiles leave O untouched), writes
-//              P_j = 2^(s - m) as bf16(P) and bf16(P - bf16(P)) into shared
-//              memory as the A operands of the P V products, and at the end
-//              writes O / l in bf16.
+//   warps 4-11 softmax: two warps per 32 query rows (TMEM lanes), one per half
+//              of the 128 key columns (and of the 128 output dims).  Each
+//              reads its half of the row of S_j, applies the scale and the
+//              causal mask, exchanges the partial row max with its partner,
+//              keeps the running max m and its half of the sum l (O is
+//              rescaled only when the max grows by more than 2^8, so most
+//              tiles leave O untouched), writes P_j = 2^(s - m) as bf16(P) and
+//              bf16(P - bf16(P)) into shared memory as the A operands of the
+//              P V products, and at the end writes its half of O / l in bf16.
 // Every wait is bounded by a deadline; one that runs out sets value 2 in the
 // caller's error word and the kernel carries on to its end.
 //
@@ -45,7 +47,7 @@ namespace {
 constexpr int kQB = 128;   // query rows per CTA (MMA M)
 constexpr int kKB = 128;   // keys per tile
 constexpr int kHD = 128;   // head dim
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;   // warp 0 TMA, warp 1 MMA, warps 4-11 softmax
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescale = 8.0f;  // O is rescaled when the running max grows by more than this (log2)
 constexpr uint64_t kDeadlineNs = 2000ull * 1000 * 1000;
@@ -193,7 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 128);
+      mbar_init(&p_full[i], 256);
     }
     mbar_init(o_done, 1);
     fence_mbar_init();
@@ -268,29 +270,45 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= 4) {
     // -------------------------------------------------------------- softmax
-    const int r = (warp - 4) * 32 + lane;  // query row of the block = TMEM lane
-    const uint32_t lane_off = (uint32_t)((warp - 4) * 32) << 16;
-    const int qpos = a.pos0 + q0 + r;      // this row sees keys 0 .. qpos
+    // Two warps per group of 32 rows (TMEM lanes): warps 4-7 take key columns
+    // 0-63 of their rows (and output dims 0-63), warps 8-11 columns 64-127.
+    // Thread r owns query row r.  The pair exchanges its partial row maxima
+    // each tile through the first 1 KB of the tile's K buffer, which S has
+    // been computed from and which is not refilled before P is published.
+    const int sw = warp - 4;                 // 0..7
+    const int rg = sw & 3, half = sw >> 2;   // lane quarter, column half
+    const int r = rg * 32 + lane;            // query row of the block = TMEM lane
+    const int cb = 64 * half;                // this warp's first column
+    const uint32_t lane_off = (uint32_t)(rg * 32) << 16;
+    const int qpos = a.pos0 + q0 + r;        // this row sees keys 0 .. qpos
     const float sl2 = a.scale * kLog2e;
+    auto softmax_sync = [] { asm volatile("bar.sync 1, 256;" ::: "memory"); };
     float m_run = -INFINITY, l_run = 0.f;
     for (int j = 0; j < nkt; ++j) {
       const int s = j & 1;
       if (!wait_bar(&s_full[s], (uint32_t)((j >> 1) & 1))) atomicOr(a.err, 2);
       fence_after();
-      // the tile's max of the scaled scores, masked beyond the row's position,
-      // 32 columns at a time (the row is read again below: short loops keep
-      // the softmax warps' code small enough to stay in the instruction cache)
-      float mt = -INFINITY;
+      // the max of this warp's half of the scaled scores, masked beyond the
+      // row's position, 32 columns at a time (the row is read again below:
+      // short loops keep the code small enough to stay in the instruction cache)
+      float mh = -INFINITY;
       const int kb = j * kKB;
 #pragma unroll 1
-      for (int c = 0; c < kKB / 32; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t sv[32];
-        tmem_ld32_nowait(tS0 + lane_off + (uint32_t)(s * kKB + 32 * c), sv);
+        tmem_ld32_nowait(tS0 + lane_off + (uint32_t)(s * kKB + cb + 32 * c), sv);
         tmem_ld_wait();
 #pragma unroll
         for (int e = 0; e < 32; ++e)
-          mt = fmaxf(mt, kb + 32 * c + e <= qpos ? __uint_as_float(sv[e]) * sl2 : -INFINITY);
+          mh = fmaxf(mh, kb + cb + 32 * c + e <= qpos ? __uint_as_float(sv[e]) * sl2 : -INFINITY);
       }
+      // the row's max: this half's and the partner's (the K buffer's TMA
+      // writes are complete: kv_full's phase is done)
+      if (!wait_bar(&kv_full[s], (uint32_t)((j >> 1) & 1))) atomicOr(a.err, 2);
+      float* xch = reinterpret_cast<float*>(smem + kKVOff + (size_t)s * kStage);
+      xch[half * kQB + r] = mh;
+      softmax_sync();
+      const float mt = fmaxf(mh, xch[(half ^ 1) * kQB + r]);
       // the product of the tile before must be done: the P buffer is reused
       // and O may be rescaled below
       if (j > 0 && !wait_bar(o_done, (uint32_t)((j - 1) & 1))) atomicOr(a.err, 2);
@@ -298,7 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // This row's max moves when the tile's max exceeds it by more than 2^8
       // (or on the first tile); O and l are then rescaled.  tcgen05.ld / st are
       // warp-collective, so the warp rescales when any of its rows needs it,
-      // the other rows by 1.
+      // the other rows by 1.  Both warps of a row take the same decision.
       float alpha = 1.f;
       if (mt > m_run + kRescale || m_run == -INFINITY) {
         const float mnew = fmaxf(mt, m_run);
@@ -308,32 +326,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       l_run *= alpha;
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
-        for (int c = 0; c < kHD / 32; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t ov[32];
-          tmem_ld32_nowait(tO + lane_off + (uint32_t)(32 * c), ov);
+          tmem_ld32_nowait(tO + lane_off + (uint32_t)(cb + 32 * c), ov);
           tmem_ld_wait();
 #pragma unroll
           for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-          tmem_st32(tO + lane_off + (uint32_t)(32 * c), ov);
+          tmem_st32(tO + lane_off + (uint32_t)(cb + 32 * c), ov);
         }
         tmem_st_wait();
       }
-      // P = 2^(s - m) as bf16 high and low parts into the K-major,
-      // 128-byte-swizzled buffers
+      // P = 2^(s - m) of this half as bf16 high and low parts into the
+      // K-major, 128-byte-swizzled buffers (this half's box)
       uint8_t* pbuf = smem + kPOff;
       const float msafe = m_run == -INFINITY ? 0.f : m_run;
       float lsum = 0.f;
 #pragma unroll 1
-      for (int c = 0; c < kKB / 32; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t sv[32];
-        tmem_ld32_nowait(tS0 + lane_off + (uint32_t)(s * kKB + 32 * c), sv);
+        tmem_ld32_nowait(tS0 + lane_off + (uint32_t)(s * kKB + cb + 32 * c), sv);
         tmem_ld_wait();
 #pragma unroll
         for (int q = 0; q < 4; ++q) {  // 16-byte chunks of 8 keys
           float pe[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const int col = 32 * c + 8 * q + e;
+            const int col = cb + 32 * c + 8 * q + e;
             const float x = kb + col <= qpos ? __uint_as_float(sv[8 * q + e]) * sl2 : -INFINITY;
             pe[e] = exp2f(x - msafe);
             lsum += pe[e];
@@ -344,8 +362,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           unpack16<bf16>(hi, phi);
 #pragma unroll
           for (int e = 0; e < 8; ++e) plo[e] = pe[e] - phi[e];
-          const int ch = 4 * c + q, box = ch >> 3, c8 = ch & 7;
-          const size_t off = box * kBox + r * 128 + ((c8 ^ (r & 7)) << 4);
+          const int c8 = 4 * c + q;  // chunk within this half's 64-key box
+          const size_t off = half * kBox + r * 128 + ((c8 ^ (r & 7)) << 4);
           *reinterpret_cast<uint4*>(pbuf + off) = hi;
           *reinterpret_cast<uint4*>(pbuf + 2 * kBox + off) = pack16<bf16>(plo);
         }
@@ -354,29 +372,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       // keys past the ones written so far are stale cache rows (possibly not
       // finite, and 0 * inf would poison the sum): zero them in V
       if (j == nkt - 1 && kb + kKB > keys_end) {
-        if (!wait_bar(&kv_full[s], (uint32_t)((j >> 1) & 1))) atomicOr(a.err, 2);
         uint8_t* vt = smem + kKVOff + (size_t)s * kStage + 2 * kBox;
         const int row0 = keys_end - kb;  // first stale row of the tile
-        for (int i = r; i < (kKB - row0) * 16; i += 128) {  // 16 chunks of 16 bytes per row
+        for (int i = sw * 32 + lane; i < (kKB - row0) * 16; i += 256) {  // 16 chunks of 16 bytes per row
           const int vr = row0 + i / 16, ch = i % 16;
           *reinterpret_cast<uint4*>(vt + (ch >> 3) * kBox + vr * 128 + (((ch & 7) ^ (vr & 7)) << 4)) =
               make_uint4(0u, 0u, 0u, 0u);
         }
       }
-      fence_proxy_async_smem();  // P (and zeroed V rows) are read by the MMA next
+      fence_proxy_async_smem();  // P, the exchange and zeroed V rows: the async proxy reads or refills them next
       fence_before();
       mbar_arrive(&p_full[s]);
     }
-    // ---- the last product, then O / l in bf16
+    // ---- the last product, then O / l in bf16: the two halves' sums are
+    // added through the P buffer (free once every product is done)
     if (nkt > 0 && !wait_bar(o_done, (uint32_t)((nkt - 1) & 1))) atomicOr(a.err, 2);
     fence_after();
-    const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+    float* lx = reinterpret_cast<float*>(smem + kPOff);
+    lx[half * kQB + r] = l_run;
+    softmax_sync();
+    const float lr = lx[r] + lx[kQB + r];
+    const float inv = lr > 0.f ? 1.f / lr : 0.f;
     const int row = q0 + r;
-    bf16* out = reinterpret_cast<bf16*>(a.out) + (size_t)row * a.out_row_stride + (size_t)h * kHD;
+    bf16* out = reinterpret_cast<bf16*>(a.out) + (size_t)row * a.out_row_stride + (size_t)h * kHD + cb;
 #pragma unroll 1
-    for (int c = 0; c < kHD / 32; ++c) {
+    for (int c = 0; c < 2; ++c) {
       uint32_t ov[32];
-      tmem_ld32_nowait(tO + lane_off + (uint32_t)(32 * c), ov);
+      tmem_ld32_nowait(tO + lane_off + (uint32_t)(cb + 32 * c), ov);
       tmem_ld_wait();
       if (row < a.rows) {
 #pragma unroll
