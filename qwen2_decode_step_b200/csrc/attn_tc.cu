@@ -12,9 +12,10 @@
 //                O   += P_j V_j   M = 128 rows, N = 128 dims, K = 128 keys,
 //                                 into TMEM O (fp32), once with P's bf16 high
 //                                 part and once with its low part (P keeps
-//                                 ~16 significant bits); V is the MN-major
-//                                 operand (dims contiguous, as the cache
-//                                 stores it)
+//                                 ~16 significant bits); P is the A operand
+//                                 in tensor memory, written over S_j's
+//                                 columns; V is the MN-major operand (dims
+//                                 contiguous, as the cache stores it)
 //              in the order S_0, S_1, O += P_0 V_0, S_2, O += P_1 V_1, ...,
 //              so a tile's scores are computed while the softmax of the tile
 //              before runs
@@ -25,8 +26,9 @@
 //              keeps the running max m and its half of the sum l (O is
 //              rescaled only when the max grows by more than 2^8, so most
 //              tiles leave O untouched), writes P_j = 2^(s - m) as bf16(P) and
-//              bf16(P - bf16(P)) into shared memory as the A operands of the
-//              P V products, and at the end writes its half of O / l in bf16.
+//              bf16(P - bf16(P)) into tensor memory over its half of S_j as
+//              the A operands of the P V products, and at the end writes its
+//              half of O / l in bf16.
 // Every wait is bounded by a deadline; one that runs out sets value 2 in the
 // caller's error word and the kernel carries on to its end.
 //
@@ -56,8 +58,7 @@ constexpr size_t kBox = (size_t)128 * 64 * 2;  // one 128-row x 64-column bf16 b
 constexpr size_t kQOff = 0;                    // Q: 2 boxes
 constexpr size_t kKVOff = 2 * kBox;            // [2 stages][K: 2 boxes | V: 2 boxes]
 constexpr size_t kStage = 4 * kBox;
-constexpr size_t kPOff = kKVOff + 2 * kStage;  // P high: 2 boxes of 128 rows x 64 keys, then P low
-constexpr size_t kBarOff = kPOff + 2 * 2 * kBox;
+constexpr size_t kBarOff = kKVOff + 2 * kStage;
 constexpr size_t kSmem = kBarOff + 16 * 8 + 16 + 1024;  // barriers, TMEM base, alignment slack
 
 __device__ __forceinline__ uint64_t gtimer() {
@@ -111,6 +112,16 @@ __device__ __forceinline__ void mma(uint32_t d_tmem, uint64_t a, uint64_t b, uin
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
       " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
       "l"(a), "l"(b), "r"(id), "r"(acc)
+      : "memory");
+}
+
+// The same with A read from tensor memory (K-major: lane = row, two bf16 of
+// consecutive k per 32-bit column).
+__device__ __forceinline__ void mma_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t id, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(id), "r"(acc)
       : "memory");
 }
 
@@ -237,18 +248,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t id_o = idesc(kHD, 1);  // O += P V: P K-major (keys contiguous), V MN-major
       const uint32_t qa = smem_u32(smem + kQOff);
       if (!wait_bar(q_full, 0)) atomicOr(a.err, 2);
-      auto pv = [&](int j) {  // O += P_j V_j
+      auto pv = [&](int j) {  // O += P_j V_j, P_j in the columns of S[j % 2]
         const int s = j & 1;
         if (!wait_bar(&p_full[s], (uint32_t)((j >> 1) & 1))) atomicOr(a.err, 2);
         fence_after();
-        const uint32_t pa = smem_u32(smem + kPOff);
+        const uint32_t tp = tS0 + (uint32_t)(s * kKB);
         const uint32_t va = smem_u32(smem + kKVOff + (size_t)s * kStage + 2 * kBox);
 #pragma unroll
         for (int k = 0; k < kKB / 16; ++k) {  // 16 keys per MMA
-          const uint32_t poff = (uint32_t)((k >> 2) * kBox) + (uint32_t)((k & 3) * 32);
+          // keys 64 hf + 16 kk ..: high part at column 64 hf + 8 kk, low part 32 further
+          const uint32_t pc = (uint32_t)(64 * (k >> 2) + 8 * (k & 3));
           const uint64_t db = desc_mnmajor(va + (uint32_t)(k * 16 * 128), (uint32_t)kBox);
-          mma(tO, desc_kmajor(pa + poff), db, id_o, (j > 0 || k > 0) ? 1u : 0u);
-          mma(tO, desc_kmajor(pa + (uint32_t)(2 * kBox) + poff), db, id_o, 1u);
+          mma_ta(tO, tp + pc, db, id_o, (j > 0 || k > 0) ? 1u : 0u);
+          mma_ta(tO, tp + pc + 32, db, id_o, 1u);
         }
         commit(o_done);
         commit(&kv_empty[s]);
@@ -309,10 +321,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       xch[half * kQB + r] = mh;
       softmax_sync();
       const float mt = fmaxf(mh, xch[(half ^ 1) * kQB + r]);
-      // the product of the tile before must be done: the P buffer is reused
-      // and O may be rescaled below
-      if (j > 0 && !wait_bar(o_done, (uint32_t)((j - 1) & 1))) atomicOr(a.err, 2);
-      fence_after();
       // This row's max moves when the tile's max exceeds it by more than 2^8
       // (or on the first tile); O and l are then rescaled.  tcgen05.ld / st are
       // warp-collective, so the warp rescales when any of its rows needs it,
@@ -325,6 +333,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       l_run *= alpha;
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        // O is rescaled once the product of the tile before is done
+        if (!wait_bar(o_done, (uint32_t)((j - 1) & 1))) atomicOr(a.err, 2);
+        fence_after();
 #pragma unroll 1
         for (int c = 0; c < 2; ++c) {
           uint32_t ov[32];
@@ -336,38 +347,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_st_wait();
       }
-      // P = 2^(s - m) of this half as bf16 high and low parts into the
-      // K-major, 128-byte-swizzled buffers (this half's box)
-      uint8_t* pbuf = smem + kPOff;
+      // P = 2^(s - m) of this half's 64 keys as bf16 high and low parts,
+      // written over this half's 64 columns of S (read first): the high parts
+      // of keys 2 e, 2 e + 1 in column e, the low parts 32 columns further.
+      // S[j % 2] is not read again, and P_j is read by the P V product before
+      // S_(j+2) is written there.
       const float msafe = m_run == -INFINITY ? 0.f : m_run;
       float lsum = 0.f;
-#pragma unroll 1
+      uint32_t phi[32], plo[32];
+#pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t sv[32];
         tmem_ld32_nowait(tS0 + lane_off + (uint32_t)(s * kKB + cb + 32 * c), sv);
         tmem_ld_wait();
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {  // 16-byte chunks of 8 keys
-          float pe[8];
+        for (int e = 0; e < 16; ++e) {
+          float pe[2];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int col = cb + 32 * c + 8 * q + e;
-            const float x = kb + col <= qpos ? __uint_as_float(sv[8 * q + e]) * sl2 : -INFINITY;
-            pe[e] = exp2f(x - msafe);
-            lsum += pe[e];
+          for (int t = 0; t < 2; ++t) {
+            const int col = cb + 32 * c + 2 * e + t;
+            const float x = kb + col <= qpos ? __uint_as_float(sv[2 * e + t]) * sl2 : -INFINITY;
+            pe[t] = exp2f(x - msafe);
+            lsum += pe[t];
           }
-          float plo[8];
-          const uint4 hi = pack16<bf16>(pe);
-          float phi[8];
-          unpack16<bf16>(hi, phi);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) plo[e] = pe[e] - phi[e];
-          const int c8 = 4 * c + q;  // chunk within this half's 64-key box
-          const size_t off = half * kBox + r * 128 + ((c8 ^ (r & 7)) << 4);
-          *reinterpret_cast<uint4*>(pbuf + off) = hi;
-          *reinterpret_cast<uint4*>(pbuf + 2 * kBox + off) = pack16<bf16>(plo);
+          const __nv_bfloat162 h2 = __floats2bfloat162_rn(pe[0], pe[1]);
+          const float2 hf = __bfloat1622float2(h2);
+          const __nv_bfloat162 l2 = __floats2bfloat162_rn(pe[0] - hf.x, pe[1] - hf.y);
+          phi[16 * c + e] = *reinterpret_cast<const uint32_t*>(&h2);
+          plo[16 * c + e] = *reinterpret_cast<const uint32_t*>(&l2);
         }
       }
+      tmem_st32(tS0 + lane_off + (uint32_t)(s * kKB + cb), phi);
+      tmem_st32(tS0 + lane_off + (uint32_t)(s * kKB + cb + 32), plo);
+      tmem_st_wait();
       l_run += lsum;
       // keys past the ones written so far are stale cache rows (possibly not
       // finite, and 0 * inf would poison the sum): zero them in V
@@ -380,15 +392,15 @@ __global__ void __launch_bounds__(kThreads, 1)
               make_uint4(0u, 0u, 0u, 0u);
         }
       }
-      fence_proxy_async_smem();  // P, the exchange and zeroed V rows: the async proxy reads or refills them next
+      fence_proxy_async_smem();  // the exchange and zeroed V rows: the async proxy refills or reads them next
       fence_before();
       mbar_arrive(&p_full[s]);
     }
     // ---- the last product, then O / l in bf16: the two halves' sums are
-    // added through the P buffer (free once every product is done)
+    // added through the Q buffer (free once every product is done)
     if (nkt > 0 && !wait_bar(o_done, (uint32_t)((nkt - 1) & 1))) atomicOr(a.err, 2);
     fence_after();
-    float* lx = reinterpret_cast<float*>(smem + kPOff);
+    float* lx = reinterpret_cast<float*>(smem + kQOff);
     lx[half * kQB + r] = l_run;
     softmax_sync();
     const float lr = lx[r] + lx[kQB + r];
