@@ -580,9 +580,12 @@ def run_profile_case(case: str):
         m.set_decode_path("stream")
         m.set_graphs(False)
         nxt = m.prefill(synth.prompt_ids(shape, 512, seed, device="cuda"), [512])
+        torch.cuda.synchronize()
+        torch.cuda.nvtx.range_push("decode")
         for _ in range(6):
             nxt = m.decode_step(nxt)
         torch.cuda.synchronize()
+        torch.cuda.nvtx.range_pop()
         m.check_error()
         m.close()
         print(f"{case}: {shape.n_layers} layers, 6 streaming steps at context 512..517")
@@ -622,9 +625,12 @@ def run_profile_case(case: str):
             m.set_seq_len(b, past)
         m.set_graphs(False)
         ids = synth.uniform_ids(B, one.vocab, wl["seed"] + 7, device="cuda")
+        torch.cuda.synchronize()
+        torch.cuda.nvtx.range_push("decode")
         for _ in range(4):
             ids = m.decode_step(ids)
         torch.cuda.synchronize()
+        torch.cuda.nvtx.range_pop()
         m.check_error()
         m.close()
         print(f"b64-layer: one decoder layer + head, batch {B}, context {past}..{past + 3}, 4 steps")
