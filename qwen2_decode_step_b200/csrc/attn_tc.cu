@@ -5,7 +5,7 @@
 //
 // One CTA per (128 query rows, query head); 384 threads:
 //   warp 0     TMA: the Q block once (two 64-dim boxes), then K and V tiles
-//              of 128 keys into a two-stage ring
+//              of 128 keys into a three-stage ring
 //   warp 1     allocates tensor memory; one thread issues the MMAs:
 //                S_j  = Q K_j^T   M = 128 rows, N = 128 keys, K = 128 dims,
 //                                 into TMEM S[j % 2] (fp32)
@@ -58,7 +58,8 @@ constexpr size_t kBox = (size_t)128 * 64 * 2;  // one 128-row x 64-column bf16 b
 constexpr size_t kQOff = 0;                    // Q: 2 boxes
 constexpr size_t kKVOff = 2 * kBox;            // [2 stages][K: 2 boxes | V: 2 boxes]
 constexpr size_t kStage = 4 * kBox;
-constexpr size_t kBarOff = kKVOff + 2 * kStage;
+constexpr int kStages = 3;                      // K/V ring depth
+constexpr size_t kBarOff = kKVOff + kStages * kStage;
 constexpr size_t kSmem = kBarOff + 16 * 8 + 16 + 1024;  // barriers, TMEM base, alignment slack
 
 __device__ __forceinline__ uint64_t gtimer() {
@@ -184,11 +185,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarOff);
   uint64_t* q_full = bars + 0;
-  uint64_t* kv_full = bars + 1;   // [2]
-  uint64_t* kv_empty = bars + 3;  // [2]
-  uint64_t* s_full = bars + 5;    // [2]
-  uint64_t* p_full = bars + 7;    // [2]
-  uint64_t* o_done = bars + 9;
+  uint64_t* kv_full = bars + 1;   // [kStages]
+  uint64_t* kv_empty = bars + 4;  // [kStages]
+  uint64_t* s_full = bars + 7;    // [2]
+  uint64_t* p_full = bars + 9;    // [2]
+  uint64_t* o_done = bars + 11;
   uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(bars + 16);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -202,9 +203,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kStages; ++i) {
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 256);
     }
@@ -231,13 +234,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int b = 0; b < 2; ++b) tma_load_2d(smem + kQOff + b * kBox, &tq, h * kHD + 64 * b, q0, q_full);
       const int xbase = kvh * a.kv_x_step, ybase = kvh * a.kv_y_step;
       for (int j = 0; j < nkt; ++j) {
-        const int s = j & 1;
-        if (j >= 2 && !wait_bar(&kv_empty[s], (uint32_t)(((j >> 1) - 1) & 1))) atomicOr(a.err, 2);
-        uint8_t* st = smem + kKVOff + s * kStage;
-        mbar_arrive_expect_tx(&kv_full[s], 4 * kBox);
+        const int kv = j % kStages;
+        if (j >= kStages && !wait_bar(&kv_empty[kv], (uint32_t)((j / kStages - 1) & 1))) atomicOr(a.err, 2);
+        uint8_t* st = smem + kKVOff + kv * kStage;
+        mbar_arrive_expect_tx(&kv_full[kv], 4 * kBox);
         for (int b = 0; b < 2; ++b) {
-          tma_load_2d(st + b * kBox, &tk, xbase + 64 * b, ybase + j * kKB, &kv_full[s]);
-          tma_load_2d(st + (2 + b) * kBox, &tv, xbase + 64 * b, ybase + j * kKB, &kv_full[s]);
+          tma_load_2d(st + b * kBox, &tk, xbase + 64 * b, ybase + j * kKB, &kv_full[kv]);
+          tma_load_2d(st + (2 + b) * kBox, &tv, xbase + 64 * b, ybase + j * kKB, &kv_full[kv]);
         }
       }
     }
@@ -249,11 +252,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t qa = smem_u32(smem + kQOff);
       if (!wait_bar(q_full, 0)) atomicOr(a.err, 2);
       auto pv = [&](int j) {  // O += P_j V_j, P_j in the columns of S[j % 2]
-        const int s = j & 1;
+        const int s = j & 1, kv = j % kStages;
         if (!wait_bar(&p_full[s], (uint32_t)((j >> 1) & 1))) atomicOr(a.err, 2);
         fence_after();
         const uint32_t tp = tS0 + (uint32_t)(s * kKB);
-        const uint32_t va = smem_u32(smem + kKVOff + (size_t)s * kStage + 2 * kBox);
+        const uint32_t va = smem_u32(smem + kKVOff + (size_t)kv * kStage + 2 * kBox);
 #pragma unroll
         for (int k = 0; k < kKB / 16; ++k) {  // 16 keys per MMA
           // keys 64 hf + 16 kk ..: high part at column 64 hf + 8 kk, low part 32 further
@@ -263,13 +266,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ta(tO, tp + pc + 32, db, id_o, 1u);
         }
         commit(o_done);
-        commit(&kv_empty[s]);
+        commit(&kv_empty[kv]);
       };
       for (int j = 0; j < nkt; ++j) {
-        const int s = j & 1;
-        if (!wait_bar(&kv_full[s], (uint32_t)((j >> 1) & 1))) atomicOr(a.err, 2);
+        const int s = j & 1, kv = j % kStages;
+        if (!wait_bar(&kv_full[kv], (uint32_t)((j / kStages) & 1))) atomicOr(a.err, 2);
         fence_after();
-        const uint32_t ka = smem_u32(smem + kKVOff + (size_t)s * kStage);
+        const uint32_t ka = smem_u32(smem + kKVOff + (size_t)kv * kStage);
 #pragma unroll
         for (int k = 0; k < kHD / 16; ++k) {  // 16 dims per MMA
           const uint32_t off = (uint32_t)((k >> 2) * kBox) + (uint32_t)((k & 3) * 32);
@@ -297,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto softmax_sync = [] { asm volatile("bar.sync 1, 256;" ::: "memory"); };
     float m_run = -INFINITY, l_run = 0.f;
     for (int j = 0; j < nkt; ++j) {
-      const int s = j & 1;
+      const int s = j & 1, kv = j % kStages;
       if (!wait_bar(&s_full[s], (uint32_t)((j >> 1) & 1))) atomicOr(a.err, 2);
       fence_after();
       // the max of this warp's half of the scaled scores, masked beyond the
@@ -316,8 +319,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // the row's max: this half's and the partner's (the K buffer's TMA
       // writes are complete: kv_full's phase is done)
-      if (!wait_bar(&kv_full[s], (uint32_t)((j >> 1) & 1))) atomicOr(a.err, 2);
-      float* xch = reinterpret_cast<float*>(smem + kKVOff + (size_t)s * kStage);
+      if (!wait_bar(&kv_full[kv], (uint32_t)((j / kStages) & 1))) atomicOr(a.err, 2);
+      float* xch = reinterpret_cast<float*>(smem + kKVOff + (size_t)kv * kStage);
       xch[half * kQB + r] = mh;
       softmax_sync();
       const float mt = fmaxf(mh, xch[(half ^ 1) * kQB + r]);
@@ -384,7 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // keys past the ones written so far are stale cache rows (possibly not
       // finite, and 0 * inf would poison the sum): zero them in V
       if (j == nkt - 1 && kb + kKB > keys_end) {
-        uint8_t* vt = smem + kKVOff + (size_t)s * kStage + 2 * kBox;
+        uint8_t* vt = smem + kKVOff + (size_t)kv * kStage + 2 * kBox;
         const int row0 = keys_end - kb;  // first stale row of the tile
         for (int i = sw * 32 + lane; i < (kKB - row0) * 16; i += 256) {  // 16 chunks of 16 bytes per row
           const int vr = row0 + i / 16, ch = i % 16;
