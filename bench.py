@@ -526,11 +526,13 @@ def prefill_gemm_rates(shape, tokens: int, peak_tflops: float, reps: int = 10):
     return out
 
 
-def long_prefill(shape, seed: int, tokens: int):
+def long_prefill(shape, seed: int, tokens: int, decode_steps: int = 64):
     """Prefill of one `tokens`-token prompt on a fresh batch-1 model (weights
-    drawn on the device), timed with CUDA events after one untimed run."""
+    drawn on the device), timed with CUDA events after one untimed run; then
+    `decode_steps` greedy decode steps over that cache (3 untimed first),
+    timed the same way."""
     import qwen2_decode_step_b200 as q2
-    m = q2.Model(shape, max_seq=tokens + 8, max_batch=1)
+    m = q2.Model(shape, max_seq=tokens + decode_steps + 8, max_batch=1)
     for key in shape.weight_shapes():
         t = synth.weight(shape, key[0], key[1], seed, device="cuda")
         m.load_weight(key[0], key[1], t)
@@ -539,9 +541,22 @@ def long_prefill(shape, seed: int, tokens: int):
     m.prefill(ids, [tokens])
     m.reset_kv()
     ms = cuda_time(lambda: m.prefill(ids, [tokens]), 1)
+    m.reset_kv()
+    nxt = m.prefill(ids, [tokens])
+    bufs = [nxt.clone(), torch.empty_like(nxt)]
+    for i in range(3):
+        m.decode_step(bufs[i % 2], out=bufs[(i + 1) % 2])
+    n = max(1, decode_steps - 3)
+    dms = cuda_time_b64(m, [bufs[1], bufs[0]], n) / n
     m.check_error()
     m.close()
-    return {"workload": WORKLOAD_LONG, "tokens": tokens, "ms": ms, "tok_s": tokens / (ms / 1e3)}
+    ctx = tokens + 3 + (n - 1) / 2.0
+    dbytes = decode_step_bytes(shape, 1, ctx)
+    hbm = float(peaks()[0]["hbm_gbs"])
+    return {"workload": WORKLOAD_LONG, "tokens": tokens, "ms": ms, "tok_s": tokens / (ms / 1e3),
+            "decode": {"steps": n, "context": f"{tokens + 3}..{tokens + 3 + n - 1}", "ms_per_step": dms,
+                       "tok_s": 1.0 / (dms / 1e3), "bytes_per_step": dbytes,
+                       "achieved_gbs": dbytes / (dms / 1e3) / 1e9, "frac": dbytes / (dms / 1e3) / 1e9 / hbm}}
 
 
 def cuda_time_b64(model, bufs, n):
