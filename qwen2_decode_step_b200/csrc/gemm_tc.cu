@@ -178,19 +178,40 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    // The weights do not depend on the kernel before this one in the stream
+    // (launched with programmatic dependent launch, this kernel may start while
+    // that one finishes): the first item's first stages get their weight boxes
+    // before the wait, their token boxes after it.
     if (lane == 0) {
       int s = 0;
       uint32_t ph = 0;
+      int early = 0;  // stages of the first item whose weight box is in flight
+      if (blockIdx.x < nitems) {
+        const int t = blockIdx.x;
+        const int tile = t % ntiles, kb0 = (t / ntiles) * a.kb_per;
+        const int kb1 = min(kblocks, kb0 + a.kb_per);
+        const int n0 = (tile % tiles_n) * kBM;
+        for (; early < STAGES && kb0 + early < kb1; ++early) {
+          mbar_arrive_expect_tx(&full[early], (uint32_t)SM::kStage);
+          tma_load_2d(smem + early * SM::kStage, &tw, (kb0 + early) * kBK, n0, &full[early]);
+        }
+      }
+      pdl_wait();
       for (int t = blockIdx.x; t < nitems; t += gridDim.x) {
         const int tile = t % ntiles, kb0 = (t / ntiles) * a.kb_per;
         const int kb1 = min(kblocks, kb0 + a.kb_per);
         const int n0 = (tile % tiles_n) * kBM, m0 = (tile / tiles_n) * BN;
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!tc_wait(&empty[s], ph ^ 1u)) atomicOr(a.err, 2);
           uint8_t* st = smem + s * SM::kStage;
-          mbar_arrive_expect_tx(&full[s], (uint32_t)SM::kStage);
-          tma_load_2d(st, &tw, kb * kBK, n0, &full[s]);
-          tma_load_2d(st + SM::kA, &tx, kb * kBK, m0, &full[s]);
+          if (early > 0) {  // the weight box is in flight: the token box
+            tma_load_2d(st + SM::kA, &tx, kb * kBK, m0, &full[s]);
+            --early;
+          } else {
+            if (!tc_wait(&empty[s], ph ^ 1u)) atomicOr(a.err, 2);
+            mbar_arrive_expect_tx(&full[s], (uint32_t)SM::kStage);
+            tma_load_2d(st, &tw, kb * kBK, n0, &full[s]);
+            tma_load_2d(st + SM::kA, &tx, kb * kBK, m0, &full[s]);
+          }
           if (++s == STAGES) {
             s = 0;
             ph ^= 1u;
@@ -231,6 +252,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    pdl_wait();  // the residual it reads and the output it writes belong to the stream's order
     const int q = warp & 3;                    // the TMEM lane quarter this warp may access
     const int half = (warp - 2) / 4;           // which alternate 32-column chunks it takes
     int it = 0;
@@ -358,7 +380,14 @@ q2_status tc_launch(const CUtensorMap& tw, const CUtensorMap& tx, const TcArgs& 
                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SM::kTotal));
   const int items = ((a.N + kBM - 1) / kBM) * ((a.M + BN - 1) / BN) * a.splits;
   const int grid = items < num_sms() ? items : num_sms();
-  tc_gemm_kernel<BN, STAGES><<<grid, kTcThreads, SM::kTotal, st>>>(tw, tx, a);
+  // programmatic dependent launch: the kernel waits (griddepcontrol.wait)
+  // before it touches anything the kernels before it produce
+  const cudaError_t le = launch_k(tc_gemm_kernel<BN, STAGES>, dim3(grid), dim3(kTcThreads), SM::kTotal, st, true,
+                                  tw, tx, a);
+  if (le != cudaSuccess) {
+    set_error(std::string("tcgen05 gemm launch: ") + cudaGetErrorString(le));
+    return Q2_ERR_CUDA;
+  }
   if (a.splits > 1) {
     const size_t total = (size_t)a.M * (a.epi == TC_EPI_SWIGLU ? a.N / 2 : a.N);
     const int blocks = (int)((total + 255) / 256 < (size_t)num_sms() * 8 ? (total + 255) / 256 : num_sms() * 8);
