@@ -51,7 +51,7 @@ __host__ __device__ inline size_t up(size_t v, size_t a) { return (v + a - 1) / 
 // the layer table has a fixed size and sits at a compile-time offset; the ring
 // (its depth is a launch parameter) and the layer table follow them.
 namespace sl {
-constexpr size_t kTiles = 0;  // [2 stages][K | V] tiles; the per-warp attention partials between items
+constexpr size_t kTiles = 0;  // [2 stages][K | V] tiles; the attention mergers' staged partials
 constexpr size_t kYrow = kTiles + 4 * (size_t)kTile;           // [kYMax] row results of a short-row phase
 constexpr size_t kPart = kYrow + (size_t)kYMax * 4;            // [kCW][kDMax] down-row column-slice sums
 constexpr size_t kXres = kPart + (size_t)kCW * kDMax * 4;       // [kDMax] this CTA's residual rows
