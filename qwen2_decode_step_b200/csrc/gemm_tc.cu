@@ -218,6 +218,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
         }
       }
+      // every load of this CTA is issued: the next kernel may start its
+      // prologue (it waits for this grid before touching its outputs)
+      pdl_launch_dependents();
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
@@ -338,6 +341,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 // then the epilogue.  One thread per output element (per gate/up pair for
 // SwiGLU).
 __global__ void tc_finish_kernel(const TcArgs a) {
+  pdl_launch_dependents();
+  pdl_wait();  // the partials are the GEMM's (launched just before it)
   const int N = a.N;
   const int cols = a.epi == TC_EPI_SWIGLU ? N / 2 : N;
   const size_t total = (size_t)a.M * cols;
@@ -391,7 +396,11 @@ q2_status tc_launch(const CUtensorMap& tw, const CUtensorMap& tx, const TcArgs& 
   if (a.splits > 1) {
     const size_t total = (size_t)a.M * (a.epi == TC_EPI_SWIGLU ? a.N / 2 : a.N);
     const int blocks = (int)((total + 255) / 256 < (size_t)num_sms() * 8 ? (total + 255) / 256 : num_sms() * 8);
-    tc_finish_kernel<<<blocks, 256, 0, st>>>(a);
+    const cudaError_t fe = launch_k(tc_finish_kernel, dim3(blocks), dim3(256), 0, st, true, a);
+    if (fe != cudaSuccess) {
+      set_error(std::string("tcgen05 gemm finish launch: ") + cudaGetErrorString(fe));
+      return Q2_ERR_CUDA;
+    }
   }
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
