@@ -306,17 +306,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the max of this warp's half of the scaled scores, masked beyond the
       // row's position, 32 columns at a time (the row is read again below:
       // short loops keep the code small enough to stay in the instruction cache)
+      // (the max of the raw scores, scaled once: scaling by a positive
+      // factor and rounding both keep the order; masking only on the tiles
+      // the block's diagonal crosses)
       float mh = -INFINITY;
       const int kb = j * kKB;
+      const bool visible = kb + kKB - 1 <= a.pos0 + q0;  // every row of the block sees the whole tile
 #pragma unroll 1
       for (int c = 0; c < 2; ++c) {
         uint32_t sv[32];
         tmem_ld32_nowait(tS0 + lane_off + (uint32_t)(s * kKB + cb + 32 * c), sv);
         tmem_ld_wait();
+        if (visible) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
-          mh = fmaxf(mh, kb + cb + 32 * c + e <= qpos ? __uint_as_float(sv[e]) * sl2 : -INFINITY);
+          for (int e = 0; e < 32; ++e) mh = fmaxf(mh, __uint_as_float(sv[e]));
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            mh = fmaxf(mh, kb + cb + 32 * c + e <= qpos ? __uint_as_float(sv[e]) : -INFINITY);
+        }
       }
+      if (mh != -INFINITY) mh *= sl2;
       // the row's max: this half's and the partner's (the K buffer's TMA
       // writes are complete: kv_full's phase is done)
       if (!wait_bar(&kv_full[kv], (uint32_t)((j / kStages) & 1))) atomicOr(a.err, 2);
@@ -355,7 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // of keys 2 e, 2 e + 1 in column e, the low parts 32 columns further.
       // S[j % 2] is not read again, and P_j is read by the P V product before
       // S_(j+2) is written there.
-      const float msafe = m_run == -INFINITY ? 0.f : m_run;
+      const float nm = m_run == -INFINITY ? 0.f : -m_run;
       float lsum = 0.f;
       uint32_t phi[32], plo[32];
 #pragma unroll
@@ -369,8 +379,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int t = 0; t < 2; ++t) {
             const int col = cb + 32 * c + 2 * e + t;
-            const float x = kb + col <= qpos ? __uint_as_float(sv[2 * e + t]) * sl2 : -INFINITY;
-            pe[t] = exp2f(x - msafe);
+            const float x = fmaf(__uint_as_float(sv[2 * e + t]), sl2, nm);
+            pe[t] = exp2f(visible || kb + col <= qpos ? x : -INFINITY);
             lsum += pe[t];
           }
           const __nv_bfloat162 h2 = __floats2bfloat162_rn(pe[0], pe[1]);
