@@ -160,6 +160,14 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// 2^x by the hardware approximation (PTX ex2.approx.ftz.f32: relative error
+// near 2^-22, results below 2^-126 flushed to zero, 2^-inf = 0)
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -303,28 +311,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int s = j & 1, kv = j % kStages;
       if (!wait_bar(&s_full[s], (uint32_t)((j >> 1) & 1))) atomicOr(a.err, 2);
       fence_after();
-      // the max of this warp's half of the scaled scores, masked beyond the
-      // row's position, 32 columns at a time (the row is read again below:
-      // short loops keep the code small enough to stay in the instruction cache)
-      // (the max of the raw scores, scaled once: scaling by a positive
-      // factor and rounding both keep the order; masking only on the tiles
-      // the block's diagonal crosses)
-      float mh = -INFINITY;
+      // This warp's half of the row's raw scores, kept in registers for both
+      // passes; keys beyond the row's position become -inf (only on the
+      // tiles the block's diagonal crosses), so 2^(s - m) is 0 there.  The
+      // max is taken over the raw scores as a tree and scaled once: scaling
+      // by a positive factor and rounding both keep the order.
       const int kb = j * kKB;
       const bool visible = kb + kKB - 1 <= a.pos0 + q0;  // every row of the block sees the whole tile
-#pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
-        uint32_t sv[32];
-        tmem_ld32_nowait(tS0 + lane_off + (uint32_t)(s * kKB + cb + 32 * c), sv);
-        tmem_ld_wait();
-        if (visible) {
+      uint32_t sv[64];
+      tmem_ld32_nowait(tS0 + lane_off + (uint32_t)(s * kKB + cb), sv);
+      tmem_ld32_nowait(tS0 + lane_off + (uint32_t)(s * kKB + cb + 32), sv + 32);
+      tmem_ld_wait();
+      if (!visible) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) mh = fmaxf(mh, __uint_as_float(sv[e]));
-        } else {
+        for (int e = 0; e < 64; ++e)
+          if (kb + cb + e > qpos) sv[e] = __float_as_uint(-INFINITY);
+      }
+      float mh;
+      {
+        float t[32];
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            mh = fmaxf(mh, kb + cb + 32 * c + e <= qpos ? __uint_as_float(sv[e]) : -INFINITY);
-        }
+        for (int e = 0; e < 32; ++e) t[e] = fmaxf(__uint_as_float(sv[e]), __uint_as_float(sv[e + 32]));
+#pragma unroll
+        for (int w = 16; w > 0; w >>= 1)
+#pragma unroll
+          for (int e = 0; e < w; ++e) t[e] = fmaxf(t[e], t[e + w]);
+        mh = t[0];
       }
       if (mh != -INFINITY) mh *= sl2;
       // the row's max: this half's and the partner's (the K buffer's TMA
@@ -361,34 +373,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_st_wait();
       }
       // P = 2^(s - m) of this half's 64 keys as bf16 high and low parts,
-      // written over this half's 64 columns of S (read first): the high parts
-      // of keys 2 e, 2 e + 1 in column e, the low parts 32 columns further.
-      // S[j % 2] is not read again, and P_j is read by the P V product before
-      // S_(j+2) is written there.
+      // written over this half's 64 columns of S: the high parts of keys
+      // 2 e, 2 e + 1 in column e, the low parts 32 columns further.  S[j % 2]
+      // is not read again, and P_j is read by the P V product before S_(j+2)
+      // is written there.
       const float nm = m_run == -INFINITY ? 0.f : -m_run;
       float lsum = 0.f;
       uint32_t phi[32], plo[32];
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t sv[32];
-        tmem_ld32_nowait(tS0 + lane_off + (uint32_t)(s * kKB + cb + 32 * c), sv);
-        tmem_ld_wait();
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          float pe[2];
-#pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            const int col = cb + 32 * c + 2 * e + t;
-            const float x = fmaf(__uint_as_float(sv[2 * e + t]), sl2, nm);
-            pe[t] = exp2f(visible || kb + col <= qpos ? x : -INFINITY);
-            lsum += pe[t];
-          }
-          const __nv_bfloat162 h2 = __floats2bfloat162_rn(pe[0], pe[1]);
-          const float2 hf = __bfloat1622float2(h2);
-          const __nv_bfloat162 l2 = __floats2bfloat162_rn(pe[0] - hf.x, pe[1] - hf.y);
-          phi[16 * c + e] = *reinterpret_cast<const uint32_t*>(&h2);
-          plo[16 * c + e] = *reinterpret_cast<const uint32_t*>(&l2);
-        }
+      for (int e = 0; e < 32; ++e) {
+        const float p0 = ex2(fmaf(__uint_as_float(sv[2 * e]), sl2, nm));
+        const float p1 = ex2(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, nm));
+        lsum += p0;
+        lsum += p1;
+        const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+        const float2 hf = __bfloat1622float2(h2);
+        const __nv_bfloat162 l2 = __floats2bfloat162_rn(p0 - hf.x, p1 - hf.y);
+        phi[e] = *reinterpret_cast<const uint32_t*>(&h2);
+        plo[e] = *reinterpret_cast<const uint32_t*>(&l2);
       }
       tmem_st32(tS0 + lane_off + (uint32_t)(s * kKB + cb), phi);
       tmem_st32(tS0 + lane_off + (uint32_t)(s * kKB + cb + 32), plo);
