@@ -12,7 +12,7 @@
 //                O   += P_j V_j   M = 128 rows, N = 128 dims, K = 128 keys,
 //                                 into TMEM O (fp32), once with P's bf16 high
 //                                 part and once with its low part (P keeps
-//                                 ~16 significant bits); P is the A operand
+//                                 16 significant bits); P is the A operand
 //                                 in tensor memory, written over S_j's
 //                                 columns; V is the MN-major operand (dims
 //                                 contiguous, as the cache stores it)
@@ -25,8 +25,8 @@
 //              causal mask, exchanges the partial row max with its partner,
 //              keeps the running max m and its half of the sum l (O is
 //              rescaled only when the max grows by more than 2^8, so most
-//              tiles leave O untouched), writes P_j = 2^(s - m) as bf16(P) and
-//              bf16(P - bf16(P)) into tensor memory over its half of S_j as
+//              tiles leave O untouched), writes P_j = 2^(s - m) as its bf16
+//              truncation hi and bf16(P - hi) into tensor memory over its half of S_j as
 //              the A operands of the P V products, and at the end writes its
 //              half of O / l in bf16.
 // Every wait is bounded by a deadline; one that runs out sets value 2 in the
@@ -305,7 +305,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = (uint32_t)(rg * 32) << 16;
     const int qpos = a.pos0 + q0 + r;        // this row sees keys 0 .. qpos
     const float sl2 = a.scale * kLog2e;
-    auto softmax_sync = [] { asm volatile("bar.sync 1, 256;" ::: "memory"); };
+    // the two warps of a row group meet on their own named barrier (1 + rg, 64 threads)
+    auto pair_sync = [rg] { asm volatile("bar.sync %0, 64;" ::"r"(1 + rg) : "memory"); };
     float m_run = -INFINITY, l_run = 0.f;
     for (int j = 0; j < nkt; ++j) {
       const int s = j & 1, kv = j % kStages;
@@ -344,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!wait_bar(&kv_full[kv], (uint32_t)((j / kStages) & 1))) atomicOr(a.err, 2);
       float* xch = reinterpret_cast<float*>(smem + kKVOff + (size_t)kv * kStage);
       xch[half * kQB + r] = mh;
-      softmax_sync();
+      pair_sync();
       const float mt = fmaxf(mh, xch[(half ^ 1) * kQB + r]);
       // This row's max moves when the tile's max exceeds it by more than 2^8
       // (or on the first tile); O and l are then rescaled.  tcgen05.ld / st are
@@ -374,24 +375,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // P = 2^(s - m) of this half's 64 keys as bf16 high and low parts,
       // written over this half's 64 columns of S: the high parts of keys
-      // 2 e, 2 e + 1 in column e, the low parts 32 columns further.  S[j % 2]
-      // is not read again, and P_j is read by the P V product before S_(j+2)
-      // is written there.
+      // 2 e, 2 e + 1 in column e, the low parts 32 columns further.  The high
+      // part is P's top 16 bits (P truncated to bf16), the low part P - high
+      // (exact in fp32, below 2^-7 P) rounded to bf16, so high + low is P to
+      // within 2^-16 of it.  S[j % 2] is not read again, and P_j is read by
+      // the P V product before S_(j+2) is written there.
       const float nm = m_run == -INFINITY ? 0.f : -m_run;
-      float lsum = 0.f;
+      float ls0 = 0.f, ls1 = 0.f;
       uint32_t phi[32], plo[32];
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
         const float p0 = ex2(fmaf(__uint_as_float(sv[2 * e]), sl2, nm));
         const float p1 = ex2(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, nm));
-        lsum += p0;
-        lsum += p1;
-        const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-        const float2 hf = __bfloat1622float2(h2);
-        const __nv_bfloat162 l2 = __floats2bfloat162_rn(p0 - hf.x, p1 - hf.y);
-        phi[e] = *reinterpret_cast<const uint32_t*>(&h2);
+        ls0 += p0;
+        ls1 += p1;
+        const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
+        phi[e] = __byte_perm(b0, b1, 0x7632);  // the upper halves: key 2 e low, key 2 e + 1 high
+        const __nv_bfloat162 l2 = __floats2bfloat162_rn(p0 - __uint_as_float(b0 & 0xFFFF0000u),
+                                                        p1 - __uint_as_float(b1 & 0xFFFF0000u));
         plo[e] = *reinterpret_cast<const uint32_t*>(&l2);
       }
+      const float lsum = ls0 + ls1;
       tmem_st32(tS0 + lane_off + (uint32_t)(s * kKB + cb), phi);
       tmem_st32(tS0 + lane_off + (uint32_t)(s * kKB + cb + 32), plo);
       tmem_st_wait();
@@ -417,7 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_after();
     float* lx = reinterpret_cast<float*>(smem + kQOff);
     lx[half * kQB + r] = l_run;
-    softmax_sync();
+    pair_sync();
     const float lr = lx[r] + lx[kQB + r];
     const float inv = lr > 0.f ? 1.f / lr : 0.f;
     const int row = q0 + r;
