@@ -380,22 +380,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       // (exact in fp32, below 2^-7 P) rounded to bf16, so high + low is P to
       // within 2^-16 of it.  S[j % 2] is not read again, and P_j is read by
       // the P V product before S_(j+2) is written there.
+      // (key pairs on the packed two-lane fp32 FMA and add: the same
+      // roundings as two scalar operations)
       const float nm = m_run == -INFINITY ? 0.f : -m_run;
-      float ls0 = 0.f, ls1 = 0.f;
+      const float2 sl2x2 = make_float2(sl2, sl2), nmx2 = make_float2(nm, nm);
+      float2 ls = make_float2(0.f, 0.f);
       uint32_t phi[32], plo[32];
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
-        const float p0 = ex2(fmaf(__uint_as_float(sv[2 * e]), sl2, nm));
-        const float p1 = ex2(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, nm));
-        ls0 += p0;
-        ls1 += p1;
-        const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
+        const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])), sl2x2, nmx2);
+        const float2 pp = make_float2(ex2(x.x), ex2(x.y));
+        ls = __fadd2_rn(ls, pp);
+        const uint32_t b0 = __float_as_uint(pp.x), b1 = __float_as_uint(pp.y);
         phi[e] = __byte_perm(b0, b1, 0x7632);  // the upper halves: key 2 e low, key 2 e + 1 high
-        const __nv_bfloat162 l2 = __floats2bfloat162_rn(p0 - __uint_as_float(b0 & 0xFFFF0000u),
-                                                        p1 - __uint_as_float(b1 & 0xFFFF0000u));
+        // minus the high parts: the top 16 bits with the sign flipped
+        const float2 lo = __fadd2_rn(pp, make_float2(__uint_as_float((b0 & 0xFFFF0000u) ^ 0x80000000u),
+                                                      __uint_as_float((b1 & 0xFFFF0000u) ^ 0x80000000u)));
+        const __nv_bfloat162 l2 = __float22bfloat162_rn(lo);
         plo[e] = *reinterpret_cast<const uint32_t*>(&l2);
       }
-      const float lsum = ls0 + ls1;
+      const float lsum = ls.x + ls.y;
       tmem_st32(tS0 + lane_off + (uint32_t)(s * kKB + cb), phi);
       tmem_st32(tS0 + lane_off + (uint32_t)(s * kKB + cb + 32), plo);
       tmem_st_wait();
