@@ -43,6 +43,17 @@ int* op_error_flag() {
   return static_cast<int*>(p);
 }
 
+// The operator entry's work-split scratch for the tensor-core attention: one
+// per device, allocated and its counters zeroed on first use, then kept.  A
+// call waits for the previous call's attention (an event) before using it, so
+// launches on different streams never share the counters at once.
+struct TcWs {
+  void* p = nullptr;
+  cudaEvent_t done = nullptr;
+};
+static std::mutex g_tcws_mu;
+static std::map<int, TcWs> g_tcws;
+
 q2_status device_error_status(int bits, const char* who) {
   std::string msg = std::string(who) + ": ";
   if (bits & kErrTimeout) {
@@ -285,7 +296,33 @@ q2_status q2_self_attention(void* out, const void* q, const void* k, const void*
   size_t bytes = attn_scratch_bytes(a.rows, a.nh, a.hd, nsplit);
   void* scratch = nullptr;
   if (bytes) Q2_CUDA_TRY(cudaMallocAsync(&scratch, bytes, st));
-  q2_status s = launch_attention(a, nsplit, scratch, dtype, st, false);
+  q2_status s;
+  if (attn_tc_supported(a, dtype)) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lk(g_tcws_mu);
+    TcWs& w = g_tcws[dev];
+    if (e == cudaSuccess && !w.p) {
+      e = cudaMalloc(&w.p, attn_tc_ws_bytes());
+      if (e == cudaSuccess) e = cudaMemsetAsync(w.p, 0, 4096, st);  // the counters
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&w.done, cudaEventDisableTiming);
+      if (e != cudaSuccess && w.p) {
+        cudaFree(w.p);
+        w.p = nullptr;
+      }
+    } else if (e == cudaSuccess) {
+      e = cudaStreamWaitEvent(st, w.done, 0);
+    }
+    if (e != cudaSuccess) {
+      if (scratch) cudaFreeAsync(scratch, st);
+      set_error(std::string("self_attention: ") + cudaGetErrorString(e));
+      return Q2_ERR_CUDA;
+    }
+    s = launch_attention(a, nsplit, scratch, dtype, st, false, nullptr, w.p);
+    cudaEventRecord(w.done, st);
+  } else {
+    s = launch_attention(a, nsplit, scratch, dtype, st, false);
+  }
   if (scratch) cudaFreeAsync(scratch, st);
   return s;
 }

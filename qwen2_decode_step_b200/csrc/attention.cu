@@ -284,14 +284,14 @@ static q2_status attn_t(const AttnRows& a, int nsplit, void* scratch, cudaStream
 }
 
 q2_status launch_attention(const AttnRows& a, int nsplit, void* scratch, int dtype,
-                           cudaStream_t st, bool pdl, int* err) {
+                           cudaStream_t st, bool pdl, int* err, void* tc_ws) {
   if (attn_tc_supported(a, dtype) && prefill_attn_impl() == 0) {
     int* e = err ? err : op_error_flag();
     if (!e) {
       set_error("attention: no error word");
       return Q2_ERR_CUDA;
     }
-    return launch_attn_tc(a, e, st);
+    return launch_attn_tc(a, tc_ws, e, st);
   }
   if (attn_prefill_mma_supported(a, dtype)) return launch_attn_prefill_mma(a, st, pdl);
   if (a.rows == 0) return Q2_OK;

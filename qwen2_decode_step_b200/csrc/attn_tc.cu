@@ -3,7 +3,18 @@
 // output accumulators in tensor memory, operands in 128-byte-swizzled shared
 // memory, K/V tiles by TMA.
 //
-// One CTA per (128 query rows, query head); 384 threads:
+// Work: an item is 128 query rows of one query head over the key tiles they
+// see (longest row blocks of each head first).  The items that fill whole
+// waves of the SMs run one CTA each; when the last, partial wave would leave
+// SMs idle, each of its items is cut instead into ts ranges of key tiles
+// (all items' first ranges first, so CTAs running together read nearby
+// keys), one CTA per range.  A range's CTA writes its partial result (O
+// unnormalised in fp32, the running max m and sum l of each row) to a slot,
+// counts itself done on the item's counter, and the range that completes the
+// count merges the item's ranges (O = sum 2^(m_k - M) O_k / sum 2^(m_k - M)
+// l_k, M = max m_k) into the bf16 rows and resets the counter.  The usual
+// write / fence / atomic pattern: no CTA waits for another.
+// One CTA per item or range; 384 threads:
 //   warp 0     TMA: the Q block once (two 64-dim boxes), then K and V tiles
 //              of 128 keys into a three-stage ring
 //   warp 1     allocates tensor memory; one thread issues the MMAs:
@@ -36,6 +47,8 @@
 // 5): scores q k^T * scale, causal mask (query i of a block at positions
 // pos0.. sees keys j <= pos0 + i), stable softmax, times V; query head h reads
 // kv head h / (nh / nkv).
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "tma.h"
@@ -182,7 +195,21 @@ struct AttnTc {
   void* out;
   long long out_row_stride;  // elements
   int* err;
+  int ntq;       // row blocks; item i is row block ntq - 1 - i % ntq of head i / ntq
+  int n_whole;   // items 0 .. n_whole - 1 run whole, one CTA each
+  int ts;        // the later items' key ranges (CTA n_whole + p: range p / n_tail of item n_whole + p % n_tail)
+  float* part;   // [n_tail * ts] slots of kSlotFloats
+  int* cnt;      // [n_tail] ranges done (0 between launches)
 };
+
+// A slot: O (fp32, [row][dim]), then m and l of each row.
+constexpr int kSlotFloats = kQB * kHD + 2 * kQB;
+
+// Key tiles of row block qt: up to the block's last visible key.
+__host__ __device__ __forceinline__ int item_tiles(int rows, int pos0, int qt) {
+  const int last_row = (qt * kQB + kQB < rows ? qt * kQB + kQB : rows) - 1;
+  return (pos0 + last_row) / kKB + 1;
+}
 
 }  // namespace
 
@@ -201,13 +228,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(bars + 16);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int ntq = (a.rows + kQB - 1) / kQB;
-  const int qt = ntq - 1 - (int)blockIdx.x;  // the longest (last) row blocks first
-  const int h = blockIdx.y, kvh = h / (a.nh / a.nkv);
+  const int n_items = a.ntq * a.nh, n_tail = n_items - a.n_whole;
+  const int piece = (int)blockIdx.x - a.n_whole;  // >= 0: a key range of a tail item
+  const int item = piece < 0 ? (int)blockIdx.x : a.n_whole + piece % n_tail;
+  const int qt = a.ntq - 1 - item % a.ntq;  // the longest (last) row blocks of a head first
+  const int h = item / a.ntq, kvh = h / (a.nh / a.nkv);
   const int q0 = qt * kQB;
-  const int last_row = min(q0 + kQB, a.rows) - 1;
-  const int nkt = (a.pos0 + last_row) / kKB + 1;  // key tiles up to the block's last visible key
-  const int keys_end = a.pos0 + a.rows;            // keys written so far (later rows are stale)
+  const int nkt = item_tiles(a.rows, a.pos0, qt);  // key tiles up to the block's last visible key
+  const int jb = piece < 0 ? 0 : (piece / n_tail) * nkt / a.ts;           // this CTA's key tiles:
+  const int n = (piece < 0 ? nkt : (piece / n_tail + 1) * nkt / a.ts) - jb;  // jb .. jb + n - 1
+  const int keys_end = a.pos0 + a.rows;  // keys written so far (later rows are stale)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -241,14 +271,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive_expect_tx(q_full, 2 * kBox);
       for (int b = 0; b < 2; ++b) tma_load_2d(smem + kQOff + b * kBox, &tq, h * kHD + 64 * b, q0, q_full);
       const int xbase = kvh * a.kv_x_step, ybase = kvh * a.kv_y_step;
-      for (int j = 0; j < nkt; ++j) {
+      for (int j = 0; j < n; ++j) {  // the CTA's j-th tile: key tile jb + j
         const int kv = j % kStages;
         if (j >= kStages && !wait_bar(&kv_empty[kv], (uint32_t)((j / kStages - 1) & 1))) atomicOr(a.err, 2);
         uint8_t* st = smem + kKVOff + kv * kStage;
         mbar_arrive_expect_tx(&kv_full[kv], 4 * kBox);
         for (int b = 0; b < 2; ++b) {
-          tma_load_2d(st + b * kBox, &tk, xbase + 64 * b, ybase + j * kKB, &kv_full[kv]);
-          tma_load_2d(st + (2 + b) * kBox, &tv, xbase + 64 * b, ybase + j * kKB, &kv_full[kv]);
+          tma_load_2d(st + b * kBox, &tk, xbase + 64 * b, ybase + (jb + j) * kKB, &kv_full[kv]);
+          tma_load_2d(st + (2 + b) * kBox, &tv, xbase + 64 * b, ybase + (jb + j) * kKB, &kv_full[kv]);
         }
       }
     }
@@ -276,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         commit(o_done);
         commit(&kv_empty[kv]);
       };
-      for (int j = 0; j < nkt; ++j) {
+      for (int j = 0; j < n; ++j) {
         const int s = j & 1, kv = j % kStages;
         if (!wait_bar(&kv_full[kv], (uint32_t)((j / kStages) & 1))) atomicOr(a.err, 2);
         fence_after();
@@ -289,7 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         commit(&s_full[s]);
         if (j > 0) pv(j - 1);
       }
-      if (nkt > 0) pv(nkt - 1);
+      if (n > 0) pv(n - 1);
     }
   } else if (warp >= 4) {
     // -------------------------------------------------------------- softmax
@@ -308,7 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the two warps of a row group meet on their own named barrier (1 + rg, 64 threads)
     auto pair_sync = [rg] { asm volatile("bar.sync %0, 64;" ::"r"(1 + rg) : "memory"); };
     float m_run = -INFINITY, l_run = 0.f;
-    for (int j = 0; j < nkt; ++j) {
+    for (int j = 0; j < n; ++j) {
       const int s = j & 1, kv = j % kStages;
       if (!wait_bar(&s_full[s], (uint32_t)((j >> 1) & 1))) atomicOr(a.err, 2);
       fence_after();
@@ -317,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // tiles the block's diagonal crosses), so 2^(s - m) is 0 there.  The
       // max is taken over the raw scores as a tree and scaled once: scaling
       // by a positive factor and rounding both keep the order.
-      const int kb = j * kKB;
+      const int kb = (jb + j) * kKB;
       const bool visible = kb + kKB - 1 <= a.pos0 + q0;  // every row of the block sees the whole tile
       uint32_t sv[64];
       tmem_ld32_nowait(tS0 + lane_off + (uint32_t)(s * kKB + cb), sv);
@@ -406,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       l_run += lsum;
       // keys past the ones written so far are stale cache rows (possibly not
       // finite, and 0 * inf would poison the sum): zero them in V
-      if (j == nkt - 1 && kb + kKB > keys_end) {
+      if (jb + j == nkt - 1 && kb + kKB > keys_end) {
         uint8_t* vt = smem + kKVOff + (size_t)kv * kStage + 2 * kBox;
         const int row0 = keys_end - kb;  // first stale row of the tile
         for (int i = sw * 32 + lane; i < (kKB - row0) * 16; i += 256) {  // 16 chunks of 16 bytes per row
@@ -419,29 +449,92 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_before();
       mbar_arrive(&p_full[s]);
     }
-    // ---- the last product, then O / l in bf16: the two halves' sums are
-    // added through the Q buffer (free once every product is done)
-    if (nkt > 0 && !wait_bar(o_done, (uint32_t)((nkt - 1) & 1))) atomicOr(a.err, 2);
+    // ---- the last product, then O / l in bf16 (or O, m, l to the range's
+    // slot): the two halves' sums are added through the Q buffer (free once
+    // every product is done)
+    if (n > 0 && !wait_bar(o_done, (uint32_t)((n - 1) & 1))) atomicOr(a.err, 2);
     fence_after();
     float* lx = reinterpret_cast<float*>(smem + kQOff);
     lx[half * kQB + r] = l_run;
     pair_sync();
     const float lr = lx[r] + lx[kQB + r];
-    const float inv = lr > 0.f ? 1.f / lr : 0.f;
     const int row = q0 + r;
     bf16* out = reinterpret_cast<bf16*>(a.out) + (size_t)row * a.out_row_stride + (size_t)h * kHD + cb;
+    if (piece < 0) {
+      const float inv = lr > 0.f ? 1.f / lr : 0.f;
 #pragma unroll 1
-    for (int c = 0; c < 2; ++c) {
-      uint32_t ov[32];
-      tmem_ld32_nowait(tO + lane_off + (uint32_t)(cb + 32 * c), ov);
-      tmem_ld_wait();
-      if (row < a.rows) {
+      for (int c = 0; c < 2; ++c) {
+        uint32_t ov[32];
+        tmem_ld32_nowait(tO + lane_off + (uint32_t)(cb + 32 * c), ov);
+        tmem_ld_wait();
+        if (row < a.rows) {
 #pragma unroll
-        for (int e = 0; e < 32; e += 8) {
-          float f[8];
+          for (int e = 0; e < 32; e += 8) {
+            float f[8];
 #pragma unroll
-          for (int t = 0; t < 8; ++t) f[t] = __uint_as_float(ov[e + t]) * inv;
-          *reinterpret_cast<uint4*>(out + 32 * c + e) = pack16<bf16>(f);
+            for (int t = 0; t < 8; ++t) f[t] = __uint_as_float(ov[e + t]) * inv;
+            *reinterpret_cast<uint4*>(out + 32 * c + e) = pack16<bf16>(f);
+          }
+        }
+      }
+    } else {
+      const int t = item - a.n_whole;
+      float* sl = a.part + (size_t)piece * kSlotFloats;
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        uint32_t ov[32];
+        tmem_ld32_nowait(tO + lane_off + (uint32_t)(cb + 32 * c), ov);
+        tmem_ld_wait();
+        float4* dst = reinterpret_cast<float4*>(sl + (size_t)r * kHD + cb + 32 * c);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          dst[e] = make_float4(__uint_as_float(ov[4 * e]), __uint_as_float(ov[4 * e + 1]),
+                               __uint_as_float(ov[4 * e + 2]), __uint_as_float(ov[4 * e + 3]));
+      }
+      sl[kQB * kHD + half * kQB + r] = half == 0 ? m_run : lr;
+      // count the range done; the one that completes the count merges
+      __threadfence();
+      int* last = reinterpret_cast<int*>(lx + 2 * kQB);
+      asm volatile("bar.sync 5, 256;" ::: "memory");
+      if (sw == 0 && lane == 0) {
+        const int done = atomicAdd(&a.cnt[t], 1);
+        if (done == a.ts - 1) a.cnt[t] = 0;  // every range has counted: ready for the next launch
+        *last = done == a.ts - 1;
+      }
+      asm volatile("bar.sync 5, 256;" ::: "memory");
+      if (*last) {
+        __threadfence();
+        float mm = -INFINITY;
+        for (int k = 0; k < a.ts; ++k)
+          mm = fmaxf(mm, __ldcg(a.part + (size_t)(k * n_tail + t) * kSlotFloats + kQB * kHD + r));
+        float o[64], ll = 0.f;
+#pragma unroll
+        for (int d = 0; d < 64; ++d) o[d] = 0.f;
+        for (int k = 0; k < a.ts; ++k) {
+          const float* sk = a.part + (size_t)(k * n_tail + t) * kSlotFloats;
+          const float mk = __ldcg(sk + kQB * kHD + r);
+          if (mk == -INFINITY) continue;  // the row sees no key in this range
+          const float w = exp2f(mk - mm);
+          ll += w * __ldcg(sk + kQB * kHD + kQB + r);
+          const float4* src = reinterpret_cast<const float4*>(sk + (size_t)r * kHD + cb);
+#pragma unroll
+          for (int d = 0; d < 16; ++d) {
+            const float4 v = __ldcg(src + d);
+            o[4 * d] += w * v.x;
+            o[4 * d + 1] += w * v.y;
+            o[4 * d + 2] += w * v.z;
+            o[4 * d + 3] += w * v.w;
+          }
+        }
+        const float inv = ll > 0.f ? 1.f / ll : 0.f;
+        if (row < a.rows) {
+#pragma unroll
+          for (int e = 0; e < 64; e += 8) {
+            float f[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) f[u] = o[e + u] * inv;
+            *reinterpret_cast<uint4*>(out + e) = pack16<bf16>(f);
+          }
         }
       }
     }
@@ -471,6 +564,11 @@ static const bf16* seq_v(const AttnRows& a) {
   return reinterpret_cast<const bf16*>(a.v) + (size_t)a.fixed_seq * a.kv_seq_stride;
 }
 
+// The work-split scratch: the tail items' counters, then their ranges' slots.
+constexpr int kMaxTs = 6;
+constexpr size_t kCntBytes = 4096;
+size_t attn_tc_ws_bytes() { return kCntBytes + (size_t)num_sms() * kMaxTs * kSlotFloats * sizeof(float); }
+
 bool attn_tc_supported(const AttnRows& a, int dtype) {
   return dtype == Q2_BF16 && a.hd == kHD && !a.seq_is_row && a.lens == nullptr && a.row_step == 1 &&
          a.nkv > 0 && a.nh % a.nkv == 0 && a.rows >= 16 && a.base >= 1 && a.fixed_seq >= 0 &&
@@ -479,7 +577,7 @@ bool attn_tc_supported(const AttnRows& a, int dtype) {
          (reinterpret_cast<uintptr_t>(seq_v(a)) & 15) == 0 && (reinterpret_cast<uintptr_t>(a.out) & 15) == 0;
 }
 
-q2_status launch_attn_tc(const AttnRows& a, int* err, cudaStream_t st) {
+q2_status launch_attn_tc(const AttnRows& a, void* ws, int* err, cudaStream_t st) {
   if (a.rows == 0) return Q2_OK;
   const int pos0 = a.base - 1;
   const long long keys = (long long)pos0 + a.rows;  // keys visible to the last row
@@ -513,9 +611,41 @@ q2_status launch_attn_tc(const AttnRows& a, int* err, cudaStream_t st) {
   p.out = a.out;
   p.out_row_stride = a.out_row_stride;
   p.err = err;
+  // The items that fill whole waves run whole; the last wave's items are cut
+  // into ts key ranges when that shortens it: with W whole waves and n_tail
+  // items left of average length len tiles, the tail takes about
+  // ceil(n_tail ts / SMs) (len / ts + c) tile times, c ~ 3 tiles for a CTA's
+  // start, pipeline fill and partial write.  ts is at most the shortest tail
+  // item's tile count.
+  p.ntq = (a.rows + kQB - 1) / kQB;
+  const int items = p.ntq * a.nh, sms = num_sms();
+  p.n_whole = items;
+  p.ts = 1;
+  p.cnt = reinterpret_cast<int*>(ws);
+  p.part = ws ? reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kCntBytes) : nullptr;
+  const int n_tail = items % sms;
+  if (ws && n_tail > 0) {
+    long long sum = 0;
+    int shortest = 1 << 30;
+    for (int i = items - n_tail; i < items; ++i) {
+      const int nt = item_tiles(a.rows, pos0, p.ntq - 1 - i % p.ntq);
+      sum += nt;
+      shortest = std::min(shortest, nt);
+    }
+    const double len = (double)sum / n_tail, c = 3.0;
+    double best = len + c;
+    for (int ts = 2; ts <= std::min(kMaxTs, shortest); ++ts) {
+      const double t = (double)((n_tail * ts + sms - 1) / sms) * (len / ts + c);
+      if (t < 0.97 * best) {
+        best = t;
+        p.ts = ts;
+      }
+    }
+    if (p.ts > 1) p.n_whole = items - n_tail;
+  }
   Q2_CUDA_TRY(cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem));
-  dim3 grid((a.rows + kQB - 1) / kQB, a.nh);
-  Q2_LAUNCH(attn_tc_kernel, grid, dim3(kThreads), kSmem, st, false, tq, tk, tv, p);
+  const int grid = p.n_whole + (items - p.n_whole) * p.ts;
+  Q2_LAUNCH(attn_tc_kernel, dim3(grid), dim3(kThreads), kSmem, st, false, tq, tk, tv, p);
   return Q2_OK;
 }
 

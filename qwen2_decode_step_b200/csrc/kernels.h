@@ -67,8 +67,11 @@ struct AttnRows {
 // Split count for a given problem (decode: enough CTAs for the machine).
 int attn_splits(int rows, int nkv, int max_keys);
 size_t attn_scratch_bytes(int rows, int nh, int hd, int nsplit);
+// tc_ws: the tensor-core path's work-split scratch (attn_tc_ws_bytes(), its
+// first 4 KB zero before the first call; the path leaves it zero), or null
+// (then every item runs whole).
 q2_status launch_attention(const AttnRows& a, int nsplit, void* scratch, int dtype,
-                           cudaStream_t st, bool pdl, int* err = nullptr);
+                           cudaStream_t st, bool pdl, int* err = nullptr, void* tc_ws = nullptr);
 // Rows of one sequence (prefill), bf16, head dim 128: flash-attention on the
 // tensor cores (launch_attention takes it by itself when it applies).
 bool attn_prefill_mma_supported(const AttnRows& a, int dtype);
@@ -78,6 +81,7 @@ q2_status launch_attn_prefill_mma(const AttnRows& a, cudaStream_t st, bool pdl);
 // out sets value 2 in *err.  launch_attention takes it when it applies.
 bool attn_tc_supported(const AttnRows& a, int dtype);
 int prefill_attn_impl();
-q2_status launch_attn_tc(const AttnRows& a, int* err, cudaStream_t st);
+size_t attn_tc_ws_bytes();
+q2_status launch_attn_tc(const AttnRows& a, void* ws, int* err, cudaStream_t st);
 
 }  // namespace q2

@@ -78,6 +78,7 @@ struct q2_model {
   int64_t* d_next = nullptr;
   float2* rope = nullptr;  // [max_seq][hd/2] (cos, sin)
   void* attn_scratch = nullptr;
+  void* attn_tc_ws = nullptr;  // the tensor-core prefill attention's work split (zeroed at creation)
   float* am_val = nullptr;
   int64_t* am_idx = nullptr;
   int* d_err = nullptr;
@@ -309,7 +310,7 @@ q2_status run_layers(q2_model* M, int T, int decode, int seq, int pos0, cudaStre
         a.fixed_seq = seq;
         nsplit = attn_splits(T, m.n_kv_heads, pos0 + T);
       }
-      TIMED(Q2_K_ATTN, launch_attention(a, nsplit, M->attn_scratch, dt, st, pdl, M->d_err));
+      TIMED(Q2_K_ATTN, launch_attention(a, nsplit, M->attn_scratch, dt, st, pdl, M->d_err, M->attn_tc_ws));
     }
 
     if (tc) {
@@ -787,6 +788,7 @@ q2_status q2_model_create(const q2_meta* meta, int device, q2_model** out) {
   al.push_back({(void**)&M->d_next, (size_t)m.max_batch * sizeof(int64_t)});
   al.push_back({(void**)&M->rope, (size_t)m.max_seq * (m.head_dim / 2) * sizeof(float2)});
   al.push_back({&M->attn_scratch, scratch});
+  if (M->dt == Q2_BF16 && m.head_dim == 128) al.push_back({&M->attn_tc_ws, attn_tc_ws_bytes()});
   al.push_back({(void**)&M->am_val, am * sizeof(float)});
   al.push_back({(void**)&M->am_idx, am * sizeof(int64_t)});
   al.push_back({(void**)&M->d_len, (size_t)m.max_batch * sizeof(int)});
