@@ -20,7 +20,10 @@ kernel's own global-timer stamps), the other decode paths' step times
 per-kernel-class breakdown), the 512-token prefill (`prefill`), the
 32768-token prefill (`prefill_long`), the tcgen05 GEMM on the prefill linears
 at 4096 tokens (the model's prefill chunk, first) and 32768 tokens
-(`prefill_gemms`, fraction of the measured bf16 peak), the host-buffer entry
+(`prefill_gemms`, fraction of the measured bf16 peak), the tcgen05 prefill
+attention on the 32768-token prompt's last chunk (`prefill_attention`: 4096
+query rows over 32768 keys, causal FLOPs over the measured bf16 peak), the
+host-buffer entry
 point end to end (`e2e`), SM clocks during the timed region (`clocks`) and
 the CPU oracle baseline (`cpu_baseline`).  Fractions of HBM are given against
 the measured copy bandwidth (`frac`) and against the ~8 TB/s datasheet
@@ -36,6 +39,7 @@ import argparse
 import datetime
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -425,6 +429,10 @@ def run_ours(args, dist: Dist):
     if not args.no_long_prefill:
         wl_long = synth.WORKLOADS[WORKLOAD_LONG]
         long_line = long_prefill(shape, wl_long["seed"] + 100 * dist.rank, wl_long["prompt"])
+    attn_rate = None
+    if not args.no_long_prefill:
+        attn_rate = prefill_attention_rate(shape, float(pk["bf16_tflops"]))
+        attn_rate["peak_kind"] = pk_kind
     if not args.no_prefill_gemms:
         gemms = {str(t): prefill_gemm_rates(shape, t, float(pk["bf16_tflops"]))
                  for t in (int(x) for x in args.prefill_gemm_tokens.split(","))}
@@ -484,6 +492,7 @@ def run_ours(args, dist: Dist):
         "kernels_per_step": kernels_per_step,
         "prefill": {"tokens": prompt_len, "ms": pre_ms, "tok_s": prompt_len / (pre_ms / 1e3)},
         "prefill_long": long_line,
+        "prefill_attention": attn_rate,
         "prefill_gemms": gemms and {"tokens": args.prefill_gemm_tokens,
                                     "peak_tflops": float(pk["bf16_tflops"]), "peak_kind": pk_kind,
                                     "kernel": "tc_gemm_kernel (tcgen05, TMEM)", "by_tokens": gemms},
@@ -524,6 +533,41 @@ def prefill_gemm_rates(shape, tokens: int, peak_tflops: float, reps: int = 10):
         del x, w, y
     q2.q2_check_device_error()
     return out
+
+
+def prefill_attention_rate(shape, peak_tflops: float, S: int = 4096, T: int = 32768, reps: int = 10):
+    """The tcgen05 prefill attention through q2_self_attention on the last
+    S-row chunk of a T-token prompt (synthetic N(0,1) bf16 q/k/v resident on
+    the device; q, k, v and out are ~59 MB for the Qwen2-1.5B shape, under
+    the 126 MB L2, so a 256 MB buffer is written between the timed calls),
+    each call timed with CUDA events on the current stream and the times
+    averaged.  FLOPs: QK^T and PV, 4 * nh * hd per visible (row, key) pair,
+    causal."""
+    import qwen2_decode_step_b200 as q2
+    nh, nkv, hd = shape.n_heads, shape.n_kv_heads, shape.head_dim
+    g = torch.Generator(device="cuda")
+    g.manual_seed(4343)
+    q = torch.randn(S, nh, hd, device="cuda", generator=g).bfloat16()
+    k = torch.randn(T, nkv, hd, device="cuda", generator=g).bfloat16()
+    v = torch.randn(T, nkv, hd, device="cuda", generator=g).bfloat16()
+    out = torch.empty(S, nh, hd, device="cuda", dtype=torch.bfloat16)
+    scale = 1.0 / math.sqrt(hd)
+    for _ in range(3):
+        q2.q2_self_attention(out, q, k, v, scale)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    ms = 0.0
+    for _ in range(reps):
+        flush.fill_(1)
+        ms += cuda_time(lambda: q2.q2_self_attention(out, q, k, v, scale), 1)
+    ms /= reps
+    del flush
+    q2.q2_check_device_error()
+    pairs = S * (T - S) + S * (S + 1) // 2
+    tf = 4.0 * nh * hd * pairs / (ms / 1e3) / 1e12
+    return {"workload": f"{S} query rows over {T} keys (the {T}-token prompt's last chunk), "
+                        f"{nh} heads / {nkv} kv heads, hd {hd}",
+            "kernel": "attn_tc_kernel (tcgen05, TMEM)", "l2": "256 MB written between timed calls",
+            "ms": ms, "tflops": tf, "frac": tf / peak_tflops}
 
 
 def long_prefill(shape, seed: int, tokens: int, decode_steps: int = 64):
