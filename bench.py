@@ -539,10 +539,11 @@ def prefill_attention_rate(shape, peak_tflops: float, S: int = 4096, T: int = 32
     """The tcgen05 prefill attention through q2_self_attention on the last
     S-row chunk of a T-token prompt (synthetic N(0,1) bf16 q/k/v resident on
     the device; q, k, v and out are ~59 MB for the Qwen2-1.5B shape, under
-    the 126 MB L2, so a 256 MB buffer is written between the timed calls),
-    each call timed with CUDA events on the current stream and the times
-    averaged.  FLOPs: QK^T and PV, 4 * nh * hd per visible (row, key) pair,
-    causal."""
+    the 126 MB L2, so a 256 MB buffer is written before every call): reps
+    back-to-back (write, call) pairs timed with CUDA events on the current
+    stream, minus reps writes alone timed the same way (the host's per-call
+    work overlaps the device's as in a prefill).  FLOPs: QK^T and PV,
+    4 * nh * hd per visible (row, key) pair, causal."""
     import qwen2_decode_step_b200 as q2
     nh, nkv, hd = shape.n_heads, shape.n_kv_heads, shape.head_dim
     g = torch.Generator(device="cuda")
@@ -555,18 +556,21 @@ def prefill_attention_rate(shape, peak_tflops: float, S: int = 4096, T: int = 32
     for _ in range(3):
         q2.q2_self_attention(out, q, k, v, scale)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
-    ms = 0.0
-    for _ in range(reps):
+
+    def flushed_call():
         flush.fill_(1)
-        ms += cuda_time(lambda: q2.q2_self_attention(out, q, k, v, scale), 1)
-    ms /= reps
+        q2.q2_self_attention(out, q, k, v, scale)
+
+    flushed_call()
+    ms = (cuda_time(flushed_call, reps) - cuda_time(lambda: flush.fill_(1), reps)) / reps
     del flush
     q2.q2_check_device_error()
     pairs = S * (T - S) + S * (S + 1) // 2
     tf = 4.0 * nh * hd * pairs / (ms / 1e3) / 1e12
     return {"workload": f"{S} query rows over {T} keys (the {T}-token prompt's last chunk), "
                         f"{nh} heads / {nkv} kv heads, hd {hd}",
-            "kernel": "attn_tc_kernel (tcgen05, TMEM)", "l2": "256 MB written between timed calls",
+            "kernel": "attn_tc_kernel (tcgen05, TMEM)",
+            "l2": "256 MB written before every call; the writes' own time subtracted",
             "ms": ms, "tflops": tf, "frac": tf / peak_tflops}
 
 
