@@ -151,7 +151,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int ntiles = tiles_n * tiles_m;
   const int nitems = ntiles * a.splits;  // (tile, K split) work items
   const int kblocks = (a.K + kBK - 1) / kBK;
-  constexpr uint32_t kCols = 2 * BN;  // two accumulators (a power of two >= 32)
+  // two accumulators of BN columns; the allocation is a power of two >= 32
+  constexpr uint32_t kCols = 2 * BN <= 32 ? 32 : 2 * BN <= 64 ? 64 : 2 * BN <= 128 ? 128 : 2 * BN <= 256 ? 256 : 512;
+  static_assert(BN % 32 == 0 && 2 * BN <= 512, "the epilogue reads 32-column chunks of two BN-column accumulators");
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
@@ -446,8 +448,17 @@ q2_status tc_gemm(void* out, int ldo, int out_dtype, int epi, const void* x, con
   a.epi = epi;
   a.err = err;
   // Token tile: 256 wide from 256 tokens up (narrower tiles fill the last
-  // wave better but double the operand traffic per FLOP; measured slower).
-  const int bn = M >= 256 ? 256 : (M >= 128 ? 128 : 64);
+  // wave better but raise the operand traffic per FLOP; 128 measured
+  // slower), 192 when that cuts the wave-quantised work by a tenth or more:
+  // ceil(tiles / SMs) x BN, e.g. 1536 features x 4096 tokens, 192 tiles of
+  // 256 (two waves, the second a third full) against 264 of 192 (two waves).
+  int bn = M >= 256 ? 256 : (M >= 128 ? 128 : 64);
+  if (bn == 256) {
+    const int sms = num_sms(), tn = (N + kBM - 1) / kBM;
+    const long long w256 = (long long)((tn * ((M + 255) / 256) + sms - 1) / sms) * 256;
+    const long long w192 = (long long)((tn * ((M + 191) / 192) + sms - 1) / sms) * 192;
+    if (10 * w192 <= 9 * w256) bn = 192;
+  }
   // Split K when the tiles alone would leave SMs idle (few output features,
   // few tokens): aim for one work item per SM, at least two k-blocks each,
   // within the workspace.
@@ -467,6 +478,7 @@ q2_status tc_gemm(void* out, int ldo, int out_dtype, int epi, const void* x, con
   Q2_TRY(make_tmap_2d_bf16(&tw, w, (uint64_t)N, (uint64_t)K, (uint64_t)K * 2, kBM, kBK, 128));
   Q2_TRY(make_tmap_2d_bf16(&tx, x, (uint64_t)M, (uint64_t)K, (uint64_t)K * 2, (uint32_t)bn, kBK, 128));
   if (bn == 256) return tc_launch<256, 4>(tw, tx, a, st);
+  if (bn == 192) return tc_launch<192, 5>(tw, tx, a, st);
   if (bn == 128) return tc_launch<128, 6>(tw, tx, a, st);
   return tc_launch<64, 8>(tw, tx, a, st);
 }

@@ -4,7 +4,10 @@ The linear of the LLAISYS report's operator list ("linear", Y = X W^T + b)
 and the two epilogues the model fuses into it (SwiGLU over interleaved
 gate/up rows, residual add).  Sizes span several 128-feature and BN-token
 tiles with ragged tails in every dimension, K not a multiple of the 64-wide
-k-block, and the token tile widths 64, 128 and 256 the kernel picks by M.
+k-block, and the token tile widths 64, 128, 192 and 256 the kernel picks by
+M and by how full the last wave of tiles is (192 wherever it cuts the
+wave-quantised work by a tenth: most of the shapes below from M = 257 up;
+the 4096-token chunks keep 256 for q/k/v and take 192 for o and down).
 """
 import pytest
 import torch
@@ -43,6 +46,27 @@ def test_tc_gemm_plain_bf16(M, N, K, bias, split):
     out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
     q2.q2_test_tc_gemm(out, cuda(x), cuda(w), cuda(b), split=split)
     assert_op_close(out, oracle.linear(x, w, b), f"tc gemm {M}x{N}x{K} split={split}")
+
+
+# The prefill chunk's products at full size, on sampled rows: both sides of
+# every 192- and 256-token tile edge the rows cross, and the last tile (4096
+# = 21 x 192 + 64: a partial 192-token tile).
+ROWS_4096 = [0, 1, 127, 128, 191, 192, 255, 256, 383, 384, 2047, 2048, 3839, 3840, 4031, 4032, 4095]
+
+
+@pytest.mark.parametrize("N,K", [
+    (2048, 1536),   # q/k/v: 256 tiles of 256 tokens (two full waves)
+    (1536, 1536),   # o: 264 tiles of 192 tokens (192 of 256 would leave the second wave a third full)
+    (1536, 8960),   # down
+])
+def test_tc_gemm_prefill_chunk_4096_sampled_rows(N, K):
+    M = 4096
+    x = normal((M, K), 1.0, 171, "bf16")
+    w = normal((N, K), 0.02, 172, "bf16")
+    out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    q2.q2_linear(out, cuda(x), cuda(w))
+    rows = torch.tensor(ROWS_4096)
+    assert_op_close(out.cpu()[rows], oracle.linear(x[rows], w, None), f"tc gemm {M}x{N}x{K} sampled rows")
 
 
 def test_tc_gemm_split_k_is_deterministic():
