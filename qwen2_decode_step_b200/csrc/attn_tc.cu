@@ -37,9 +37,10 @@
 //              keeps the running max m and its half of the sum l (O is
 //              rescaled only when the max grows by more than 2^8, so most
 //              tiles leave O untouched), writes P_j = 2^(s - m) as its bf16
-//              truncation hi and bf16(P - hi) into tensor memory over its half of S_j as
-//              the A operands of the P V products, and at the end writes its
-//              half of O / l in bf16.
+//              truncation hi and bf16(P - hi) into tensor memory over its
+//              half of S_j as the A operands of the P V products, and at the
+//              end writes its half of O / l in bf16 (a key range: O, m and l
+//              to the range's slot, then the counter and perhaps the merge).
 // Every wait is bounded by a deadline; one that runs out sets value 2 in the
 // caller's error word and the kernel carries on to its end.
 //
@@ -69,7 +70,7 @@ constexpr uint64_t kDeadlineNs = 2000ull * 1000 * 1000;
 
 constexpr size_t kBox = (size_t)128 * 64 * 2;  // one 128-row x 64-column bf16 box: 16 KB
 constexpr size_t kQOff = 0;                    // Q: 2 boxes
-constexpr size_t kKVOff = 2 * kBox;            // [2 stages][K: 2 boxes | V: 2 boxes]
+constexpr size_t kKVOff = 2 * kBox;            // [kStages][K: 2 boxes | V: 2 boxes]
 constexpr size_t kStage = 4 * kBox;
 constexpr int kStages = 3;                      // K/V ring depth
 constexpr size_t kBarOff = kKVOff + kStages * kStage;
