@@ -78,6 +78,19 @@ q2_status q2_check_device_error(void* stream);
  * Synchronises. */
 q2_status q2_test_raise_device_error(int bits, void* stream);
 
+/* Test hook: the host-side work plans of the tensor-core kernels for a
+ * machine of `sms` SMs (no device is touched).
+ * q2_test_attn_plan: the tcgen05 prefill attention of `rows` query rows at
+ * positions pos0.. with nh query heads (128-row items of one head, each
+ * head's longest first): out[0] items run whole, out[1] key ranges ts per
+ * later item, out[2] CTAs launched, out[3] items, out[4] range slots the
+ * scratch holds, out[5] item counters it holds.  Q2_ERR_INVALID_ARG for
+ * NULL out, rows, nh or sms of 0, or sizes past 2^30.
+ * q2_test_gemm_tile: the token tile width (64, 128, 192 or 256) the tcgen05
+ * GEMM takes for M tokens x N features, in *bn. */
+q2_status q2_test_attn_plan(size_t rows, size_t pos0, size_t nh, int sms, int* out);
+q2_status q2_test_gemm_tile(size_t M, size_t N, int sms, int* bn);
+
 /* ======================================================================== */
 /* Operators (report section 3.2, third layer).  Device pointers, caller-   */
 /* owned; asynchronous on `stream`.                                          */

@@ -19,7 +19,8 @@ import torch
 
 __all__ = [
     "Q2Error", "lib", "q2_version", "q2_check_device_error", "q2_add", "q2_argmax",
-    "q2_argmax_noalloc", "q2_embedding", "q2_test_raise_device_error",
+    "q2_argmax_noalloc", "q2_embedding", "q2_test_raise_device_error", "q2_test_attn_plan",
+    "q2_test_gemm_tile",
     "q2_linear", "q2_test_tc_gemm", "q2_rms_norm", "q2_add_rms_norm", "q2_rope", "q2_self_attention", "q2_swiglu",
     "q2_rearrange", "Model", "W_KIND", "STATUS", "KCLASS",
 ]
@@ -85,6 +86,8 @@ _SIGS = {
     "q2_model_head": [_VP, _VP, _I, _VP, _VP, _VP],
     "q2_model_set_decode_path": [_VP, _I],
     "q2_test_raise_device_error": [_I, _VP],
+    "q2_test_attn_plan": [_SZ, _SZ, _SZ, _I, _VP],
+    "q2_test_gemm_tile": [_SZ, _SZ, _I, _VP],
     "q2_test_model_raise_error": [_VP, _I, _VP],
     "q2_test_set_wait_fault": [_VP, _I, ctypes.c_ulonglong],
     "q2_test_trace_stream_step": [_VP, _VP, _VP, _SZ, ctypes.POINTER(_I), _VP],
@@ -161,6 +164,22 @@ def q2_check_device_error() -> None:
 def q2_test_raise_device_error(bits: int) -> None:
     """Test hook: OR `bits` into the operators' device error word."""
     _call("q2_test_raise_device_error", bits, _stream())
+
+
+def q2_test_attn_plan(rows: int, pos0: int, nh: int, sms: int) -> dict:
+    """Test hook: the tcgen05 prefill attention's work plan on a machine of
+    `sms` SMs (host only, no device)."""
+    out = (ctypes.c_int * 6)()
+    _call("q2_test_attn_plan", rows, pos0, nh, sms, ctypes.cast(out, _VP))
+    keys = ("n_whole", "ts", "ctas", "items", "slot_capacity", "counter_capacity")
+    return dict(zip(keys, list(out)))
+
+
+def q2_test_gemm_tile(M: int, N: int, sms: int) -> int:
+    """Test hook: the token tile width the tcgen05 GEMM takes for M x N (host only)."""
+    bn = ctypes.c_int(0)
+    _call("q2_test_gemm_tile", M, N, sms, ctypes.cast(ctypes.pointer(bn), _VP))
+    return bn.value
 
 
 def q2_add(c, a, b):

@@ -111,6 +111,32 @@ q2_status q2_check_device_error(void* stream) {
   return Q2_OK;
 }
 
+q2_status q2_test_attn_plan(size_t rows, size_t pos0, size_t nh, int sms, int* out) {
+  clear_error();
+  Q2_CHECK_ARG(out && rows > 0 && nh > 0 && sms > 0, Q2_ERR_INVALID_ARG,
+               "test_attn_plan: NULL out, or rows, nh or sms of 0");
+  Q2_CHECK_ARG(rows < (1u << 30) && pos0 < (1u << 30) && nh < (1u << 16) && sms < (1 << 16),
+               Q2_ERR_INVALID_ARG, "test_attn_plan: size too large");
+  int n_whole = 0, ts = 0;
+  attn_tc_plan((int)rows, (int)pos0, (int)nh, sms, true, &n_whole, &ts);
+  const int items = (int)((rows + 127) / 128 * nh);
+  out[0] = n_whole;
+  out[1] = ts;
+  out[2] = n_whole + (items - n_whole) * ts;
+  out[3] = items;
+  out[4] = attn_tc_slot_capacity(sms);
+  out[5] = attn_tc_counter_capacity();
+  return Q2_OK;
+}
+
+q2_status q2_test_gemm_tile(size_t M, size_t N, int sms, int* bn) {
+  clear_error();
+  Q2_CHECK_ARG(bn && M > 0 && N > 0 && sms > 0 && M < (1u << 30) && N < (1u << 30), Q2_ERR_INVALID_ARG,
+               "test_gemm_tile: NULL bn, sizes of 0 or past 2^30, or no SMs");
+  *bn = tc_gemm_token_tile((int)M, (int)N, sms);
+  return Q2_OK;
+}
+
 q2_status q2_test_raise_device_error(int bits, void* stream) {
   clear_error();
   Q2_CHECK_ARG(bits > 0 && bits <= (kErrIndex | kErrTimeout), Q2_ERR_INVALID_ARG,

@@ -570,6 +570,41 @@ constexpr int kMaxTs = 6;
 constexpr size_t kCntBytes = 4096;
 size_t attn_tc_ws_bytes() { return kCntBytes + (size_t)num_sms() * kMaxTs * kSlotFloats * sizeof(float); }
 
+int attn_tc_slot_capacity(int sms) { return sms * kMaxTs; }
+int attn_tc_counter_capacity() { return (int)(kCntBytes / sizeof(int)); }
+
+// The items that fill whole waves run whole; the last wave's items are cut
+// into ts key ranges when that shortens it: with n_tail items left of average
+// length len tiles, the tail takes about ceil(n_tail ts / SMs) (len / ts + c)
+// tile times, c ~ 3 tiles for a CTA's start, pipeline fill and partial write;
+// a ts is taken only if it saves 3 %.  ts is at most kMaxTs and the shortest
+// tail item's tile count (every range has a tile); n_tail < SMs, so the
+// ranges fit SMs x kMaxTs slots.
+void attn_tc_plan(int rows, int pos0, int nh, int sms, bool split_ok, int* n_whole, int* ts) {
+  const int ntq = (rows + kQB - 1) / kQB, items = ntq * nh;
+  *n_whole = items;
+  *ts = 1;
+  const int n_tail = items % sms;
+  if (!split_ok || n_tail == 0) return;
+  long long sum = 0;
+  int shortest = 1 << 30;
+  for (int i = items - n_tail; i < items; ++i) {
+    const int nt = item_tiles(rows, pos0, ntq - 1 - i % ntq);
+    sum += nt;
+    shortest = std::min(shortest, nt);
+  }
+  const double len = (double)sum / n_tail, c = 3.0;
+  double best = len + c;
+  for (int t = 2; t <= std::min(kMaxTs, shortest); ++t) {
+    const double cost = (double)((n_tail * t + sms - 1) / sms) * (len / t + c);
+    if (cost < 0.97 * best) {
+      best = cost;
+      *ts = t;
+    }
+  }
+  if (*ts > 1) *n_whole = items - n_tail;
+}
+
 bool attn_tc_supported(const AttnRows& a, int dtype) {
   return dtype == Q2_BF16 && a.hd == kHD && !a.seq_is_row && a.lens == nullptr && a.row_step == 1 &&
          a.nkv > 0 && a.nh % a.nkv == 0 && a.rows >= 16 && a.base >= 1 && a.fixed_seq >= 0 &&
@@ -612,38 +647,11 @@ q2_status launch_attn_tc(const AttnRows& a, void* ws, int* err, cudaStream_t st)
   p.out = a.out;
   p.out_row_stride = a.out_row_stride;
   p.err = err;
-  // The items that fill whole waves run whole; the last wave's items are cut
-  // into ts key ranges when that shortens it: with W whole waves and n_tail
-  // items left of average length len tiles, the tail takes about
-  // ceil(n_tail ts / SMs) (len / ts + c) tile times, c ~ 3 tiles for a CTA's
-  // start, pipeline fill and partial write.  ts is at most the shortest tail
-  // item's tile count.
   p.ntq = (a.rows + kQB - 1) / kQB;
-  const int items = p.ntq * a.nh, sms = num_sms();
-  p.n_whole = items;
-  p.ts = 1;
+  const int items = p.ntq * a.nh;
+  attn_tc_plan(a.rows, pos0, a.nh, num_sms(), ws != nullptr, &p.n_whole, &p.ts);
   p.cnt = reinterpret_cast<int*>(ws);
   p.part = ws ? reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kCntBytes) : nullptr;
-  const int n_tail = items % sms;
-  if (ws && n_tail > 0) {
-    long long sum = 0;
-    int shortest = 1 << 30;
-    for (int i = items - n_tail; i < items; ++i) {
-      const int nt = item_tiles(a.rows, pos0, p.ntq - 1 - i % p.ntq);
-      sum += nt;
-      shortest = std::min(shortest, nt);
-    }
-    const double len = (double)sum / n_tail, c = 3.0;
-    double best = len + c;
-    for (int ts = 2; ts <= std::min(kMaxTs, shortest); ++ts) {
-      const double t = (double)((n_tail * ts + sms - 1) / sms) * (len / ts + c);
-      if (t < 0.97 * best) {
-        best = t;
-        p.ts = ts;
-      }
-    }
-    if (p.ts > 1) p.n_whole = items - n_tail;
-  }
   Q2_CUDA_TRY(cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem));
   const int grid = p.n_whole + (items - p.n_whole) * p.ts;
   Q2_LAUNCH(attn_tc_kernel, dim3(grid), dim3(kThreads), kSmem, st, false, tq, tk, tv, p);

@@ -421,6 +421,20 @@ bool tc_linear_supported(int M, int N, int K, const void* out, const void* in, c
   return (al & 15) == 0;
 }
 
+// Token tile: 256 wide from 256 tokens up (narrower tiles fill the last wave
+// better but raise the operand traffic per FLOP; 128 measured slower), 192
+// when that cuts the wave-quantised work by a tenth or more: ceil(tiles /
+// SMs) x BN, e.g. 1536 features x 4096 tokens, 192 tiles of 256 (two waves,
+// the second a third full) against 264 of 192 (two waves).
+int tc_gemm_token_tile(int M, int N, int sms) {
+  if (M < 128) return 64;
+  if (M < 256) return 128;
+  const long long tn = (N + kBM - 1) / kBM;
+  const long long w256 = (tn * ((M + 255) / 256) + sms - 1) / sms * 256;
+  const long long w192 = (tn * ((M + 191) / 192) + sms - 1) / sms * 192;
+  return 10 * w192 <= 9 * w256 ? 192 : 256;
+}
+
 q2_status tc_gemm(void* out, int ldo, int out_dtype, int epi, const void* x, const void* w,
                   const void* bias, int M, int N, int K, cudaStream_t st, int* err, float* ws,
                   size_t ws_bytes) {
@@ -447,18 +461,7 @@ q2_status tc_gemm(void* out, int ldo, int out_dtype, int epi, const void* x, con
   a.out_f32 = out_dtype == Q2_F32;
   a.epi = epi;
   a.err = err;
-  // Token tile: 256 wide from 256 tokens up (narrower tiles fill the last
-  // wave better but raise the operand traffic per FLOP; 128 measured
-  // slower), 192 when that cuts the wave-quantised work by a tenth or more:
-  // ceil(tiles / SMs) x BN, e.g. 1536 features x 4096 tokens, 192 tiles of
-  // 256 (two waves, the second a third full) against 264 of 192 (two waves).
-  int bn = M >= 256 ? 256 : (M >= 128 ? 128 : 64);
-  if (bn == 256) {
-    const int sms = num_sms(), tn = (N + kBM - 1) / kBM;
-    const long long w256 = (long long)((tn * ((M + 255) / 256) + sms - 1) / sms) * 256;
-    const long long w192 = (long long)((tn * ((M + 191) / 192) + sms - 1) / sms) * 192;
-    if (10 * w192 <= 9 * w256) bn = 192;
-  }
+  const int bn = tc_gemm_token_tile(M, N, num_sms());
   // Split K when the tiles alone would leave SMs idle (few output features,
   // few tokens): aim for one work item per SM, at least two k-blocks each,
   // within the workspace.

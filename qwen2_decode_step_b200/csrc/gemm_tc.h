@@ -17,6 +17,10 @@ enum { TC_EPI_PLAIN = 0, TC_EPI_SWIGLU = 1, TC_EPI_RESID = 2 };
 // Whether the tcgen05 path takes this linear (bf16 operands, M >= 64 tokens,
 // N >= 128 features, K a multiple of 8, operands 16-byte aligned).
 bool tc_linear_supported(int M, int N, int K, const void* out, const void* in, const void* w);
+// The token tile width (BN) tc_gemm takes for M tokens x N features on a
+// machine of `sms` SMs: 64 or 128 below 256 tokens, else 256, or 192 where
+// that cuts ceil(tiles / sms) x BN by a tenth.  Host only.
+int tc_gemm_token_tile(int M, int N, int sms);
 // out[M, N] (out_dtype) = in[M, K] . w[N, K]^T (+ bias[N]), bf16 operands.
 // A pipeline wait that runs out sets value 2 in the operators' error word.
 q2_status tc_linear(void* out, const void* in, const void* w, const void* bias, int M, int N, int K,

@@ -82,6 +82,14 @@ q2_status launch_attn_prefill_mma(const AttnRows& a, cudaStream_t st, bool pdl);
 bool attn_tc_supported(const AttnRows& a, int dtype);
 int prefill_attn_impl();
 size_t attn_tc_ws_bytes();
+// Its work plan (host only; `sms` the machine's SM count): of the
+// ceil(rows / 128) * nh items (128 query rows of one head), the first
+// *n_whole run whole, one CTA each, and each later item as *ts key ranges;
+// with !split_ok (no scratch) every item runs whole.  The scratch holds
+// attn_tc_slot_capacity(sms) ranges and attn_tc_counter_capacity() items.
+void attn_tc_plan(int rows, int pos0, int nh, int sms, bool split_ok, int* n_whole, int* ts);
+int attn_tc_slot_capacity(int sms);
+int attn_tc_counter_capacity();
 q2_status launch_attn_tc(const AttnRows& a, void* ws, int* err, cudaStream_t st);
 
 }  // namespace q2
